@@ -1,0 +1,242 @@
+/*
+ * hashgrid_oracle.c -- plain, slow, CPU-only oracle for the multiresolution hash-grid
+ * encoding (Instant-NGP style), forward and backward.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check of the package entry file and
+ * the CPU-baseline leg of the benchmark may load or call this code. The CUDA library shares
+ * no code, header, table or constant with it, and neither side includes the other.
+ *
+ * Sources, cited by page and section (the pages are web articles; they print no worked
+ * numbers, so every check of this file is self-made, see the test suite):
+ *   [NeRFace-HG]  "NeRFace + Instant-NGP hash encoding" article (ipipp.com, 0929/63223),
+ *                 section 2 (二, multiresolution feature grids): per-level table of T
+ *                 F-wide learnable features, resolution growing geometrically from N_min to
+ *                 N_max, voxel of x with its 8 corners, corner hash, trilinear interpolation,
+ *                 concatenation of the L levels into an L*F vector; the backward pass only
+ *                 updates the sampled features (end of section 2 and section 3, 三).
+ *   [Repro-HG]    "Reproduce Instant-NGP's hash-encoding layer in PyTorch" (jsqmd.com,
+ *                 news/998204): section 2.1 (level table: coarsest 16^3, finest 512^3,
+ *                 T = 2^19, F = 2), section 2.2 (hash = XOR over axes of coordinate times a
+ *                 per-axis prime, modulo T), section 3 (the layer), section 5 (half-precision
+ *                 tables to save memory).
+ *   [Overview-HG] Instant-NGP overview (ijyty.com, news/1538821), section 2.2: the hash
+ *                 h(x) = (XOR_i x_i * pi_i) mod T.
+ *
+ * Readings taken where the pages are silent or disagree (each one is listed in the design
+ * notes of the repository):
+ *   - resolution: N_l is the exact-math value of N_min * b^l, floored (R1 below);
+ *   - the point is scaled by N_l, not N_l - 1 (the NeRFace article's reading);
+ *   - the hash is evaluated in unsigned 32-bit wraparound arithmetic; for a power-of-two T
+ *     the "mod T" of the pages' 64-bit products keeps the same low bits;
+ *   - every level is hashed, including coarse levels whose vertices would fit in T;
+ *   - the offset along axis i is weighted by frac_i (true trilinear interpolation); the
+ *     pages' own snippets pair the x fraction with the z offset, which is not trilinear;
+ *   - the point is scaled in fp32 (the pages scale an fp32 coordinate tensor), so the voxel
+ *     decision x*N_l -> floor is taken in fp32 on both sides; everything after that here
+ *     is fp64.
+ *
+ * Corner numbering (shared convention of the C ABI, not arithmetic): corner c in 0..7 has
+ * offsets d0 = c & 1 (x), d1 = (c >> 1) & 1 (y), d2 = (c >> 2) & 1 (z).
+ *
+ * Table layout: table[l][i][f] at element (l*T + i)*F + f.  Output layout: out[p][l*F + f].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_PRIME_X 1u
+#define ORACLE_PRIME_Y 2654435761u
+#define ORACLE_PRIME_Z 805459861u
+
+/* ------------------------------------------------------------------------------------ */
+/* Resolution schedule.                                                                   */
+/* [NeRFace-HG] section 2: b = exp((ln N_max - ln N_min)/(L - 1)), N_l = floor(N_min b^l). */
+/* [Repro-HG] section 2.1 prints 16^3 for the coarsest and 512^3 for the finest level.     */
+/* R1: computed literally in double, N_min*b^l can land a few ulp below an integer that    */
+/* it equals in exact arithmetic (16*b^15 = 4095.99999... for N_max = 4096), and the floor */
+/* then loses one. The reading taken: when v is within 1e-9*v of an integer, that integer  */
+/* is the exact value and is used; otherwise floor(v). With L = 1 the formula divides by   */
+/* zero; the reading taken is b = 1, allowed only when N_min == N_max.                     */
+/* Returns 0 on success, -1 on invalid arguments.                                          */
+/* ------------------------------------------------------------------------------------ */
+int oracle_resolutions(int L, int N_min, int N_max, int *res)
+{
+    if (L < 1 || N_min < 1 || N_max < N_min || res == NULL)
+        return -1;
+    if (L == 1) {
+        if (N_min != N_max)
+            return -1;
+        res[0] = N_min;
+        return 0;
+    }
+    double b = exp((log((double)N_max) - log((double)N_min)) / (double)(L - 1));
+    for (int l = 0; l < L; ++l) {
+        double v = (double)N_min * pow(b, (double)l);
+        double r = nearbyint(v);
+        if (fabs(v - r) <= 1e-9 * v)
+            res[l] = (int)r;
+        else
+            res[l] = (int)floor(v);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Spatial hash of one integer vertex.                                                    */
+/* [NeRFace-HG] section 2 and [Repro-HG] section 2.2: each coordinate is multiplied by its */
+/* axis prime (1, 2654435761, 805459861) and the products are XORed. [Overview-HG] §2.2    */
+/* writes the same formula. Coordinates are taken modulo 2^32 (two's complement for        */
+/* negative vertices) and the products wrap at 2^32.                                      */
+/* ------------------------------------------------------------------------------------ */
+uint32_t oracle_hash3(int64_t c0, int64_t c1, int64_t c2)
+{
+    uint32_t u0 = (uint32_t)c0, u1 = (uint32_t)c1, u2 = (uint32_t)c2;
+    return (u0 * ORACLE_PRIME_X) ^ (u1 * ORACLE_PRIME_Y) ^ (u2 * ORACLE_PRIME_Z);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* IEEE 754 binary16 -> double, from the format's definition (1 sign bit, 5 exponent bits */
+/* with bias 15, 10 fraction bits; exponent 0 = subnormal m * 2^-24; exponent 31 = inf or */
+/* NaN). [Repro-HG] section 5 suggests half-precision tables; their values are decoded     */
+/* exactly here (every binary16 value is exact in double).                                 */
+/* ------------------------------------------------------------------------------------ */
+double oracle_half_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else if (e == 31)
+        v = (m == 0) ? INFINITY : NAN;
+    else
+        v = ldexp((double)(1024 + m), e - 25);
+    return sign ? -v : v;
+}
+
+/* Table element as double. dtype 0 = fp32, 1 = fp16 bits. */
+static double table_value(const void *table, int dtype, size_t elem)
+{
+    if (dtype == 0)
+        return (double)((const float *)table)[elem];
+    return oracle_half_to_double(((const uint16_t *)table)[elem]);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Voxel and fraction of one point at one level.                                         */
+/* [NeRFace-HG] section 2: the point is scaled by the level's resolution, floored to the  */
+/* voxel's lower vertex, and the remainder is the position inside the voxel. The scaling  */
+/* is one fp32 multiply (the pages scale an fp32 tensor); the remainder xs - floor(xs) is */
+/* exact in fp32.                                                                         */
+/* ------------------------------------------------------------------------------------ */
+static void locate(const float *xp, int res_l, int64_t v[3], double frac[3])
+{
+    for (int i = 0; i < 3; ++i) {
+        float xs = xp[i] * (float)res_l;
+        float fl = floorf(xs);
+        v[i] = (int64_t)fl;
+        frac[i] = (double)(xs - fl);
+    }
+}
+
+/* Corner c of the voxel: its vertex and its trilinear weight (product over axes of       */
+/* frac_i for offset 1 and 1 - frac_i for offset 0), [NeRFace-HG] section 2.              */
+static double corner(const int64_t v[3], const double frac[3], int c, int64_t vc[3])
+{
+    double w = 1.0;
+    for (int i = 0; i < 3; ++i) {
+        int d = (c >> i) & 1;
+        vc[i] = v[i] + d;
+        w *= d ? frac[i] : 1.0 - frac[i];
+    }
+    return w;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Hash indices of every corner: idx[p][l][c] = hash(corner) mod T, T = 2^log2T.          */
+/* Levels l0 <= l < l1 are written; idx has room for all L levels per point.             */
+/* ------------------------------------------------------------------------------------ */
+void oracle_indices(int L, int log2T, const int *res, const float *x, int64_t N,
+                    int l0, int l1, uint32_t *idx)
+{
+    uint32_t mask = (uint32_t)((1ull << log2T) - 1ull);
+    for (int64_t p = 0; p < N; ++p) {
+        for (int l = l0; l < l1; ++l) {
+            int64_t v[3], vc[3];
+            double frac[3];
+            locate(x + 3 * p, res[l], v, frac);
+            for (int c = 0; c < 8; ++c) {
+                (void)corner(v, frac, c, vc);
+                idx[((size_t)p * L + l) * 8 + c] = oracle_hash3(vc[0], vc[1], vc[2]) & mask;
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Forward pass. [NeRFace-HG] section 2 and [Repro-HG] section 3:                         */
+/*   out[p][l*F + f] = sum_c w_c * table[l][hash(corner_c) mod T][f]                      */
+/* with the sum and weights in fp64. Levels l0 <= l < l1 are written (the rest of out is */
+/* untouched). Parallel over points when nthreads > 1: every point is independent, so    */
+/* the result does not depend on the thread count.                                        */
+/* ------------------------------------------------------------------------------------ */
+void oracle_forward(int L, int F, int log2T, const int *res, int dtype, const void *table,
+                    const float *x, int64_t N, int l0, int l1, double *out, int nthreads)
+{
+    size_t T = (size_t)1 << log2T;
+    uint32_t mask = (uint32_t)(T - 1);
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+    for (int64_t p = 0; p < N; ++p) {
+        for (int l = l0; l < l1; ++l) {
+            int64_t v[3], vc[3];
+            double frac[3];
+            double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            locate(x + 3 * p, res[l], v, frac);
+            for (int c = 0; c < 8; ++c) {
+                double w = corner(v, frac, c, vc);
+                uint32_t h = oracle_hash3(vc[0], vc[1], vc[2]) & mask;
+                for (int f = 0; f < F; ++f)
+                    acc[f] += w * table_value(table, dtype, ((size_t)l * T + h) * F + f);
+            }
+            for (int f = 0; f < F; ++f)
+                out[(size_t)p * L * F + (size_t)l * F + f] = acc[f];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Backward pass with respect to the tables. The forward pass is linear in the table, so */
+/* each corner passes its weight times the upstream gradient to the entry it read; only  */
+/* the sampled entries receive gradient ([NeRFace-HG] end of section 2 and section 3).   */
+/*   dtable[l][hash(corner_c) mod T][f] += w_c * g[p][l*F + f]                            */
+/* Accumulates into dtable (fp64, caller zeroes it). Within one level the order is p, c. */
+/* Levels are disjoint slices, so running levels on separate threads gives the same bits */
+/* as a serial run.                                                                      */
+/* ------------------------------------------------------------------------------------ */
+void oracle_backward(int L, int F, int log2T, const int *res, const float *x, const float *g,
+                     int64_t N, int l0, int l1, double *dtable, int nthreads)
+{
+    size_t T = (size_t)1 << log2T;
+    uint32_t mask = (uint32_t)(T - 1);
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int l = l0; l < l1; ++l) {
+        for (int64_t p = 0; p < N; ++p) {
+            int64_t v[3], vc[3];
+            double frac[3];
+            locate(x + 3 * p, res[l], v, frac);
+            for (int c = 0; c < 8; ++c) {
+                double w = corner(v, frac, c, vc);
+                uint32_t h = oracle_hash3(vc[0], vc[1], vc[2]) & mask;
+                for (int f = 0; f < F; ++f)
+                    dtable[((size_t)l * T + h) * F + f] +=
+                        w * (double)g[(size_t)p * L * F + (size_t)l * F + f];
+            }
+        }
+    }
+}

@@ -1,0 +1,65 @@
+"""Planted mistakes: each mutation below is a plausible bug in the oracle's arithmetic,
+applied to a temporary copy of its C source and built on the CPU. The pins of
+``test_oracle_pins.py`` are then run against the mutant; at least one must fail. This
+shows the pins constrain every part of the oracle (hash, resolution, axis pairing,
+weights, corner count, accumulation), not just the parts they were written for.
+"""
+import ctypes
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+import tests.test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "hashgrid_oracle.c")
+
+MUTATIONS = {
+    # x fraction paired with the z offset, as in the pages' own snippets
+    "axis_swap": ("w *= d ? frac[i] : 1.0 - frac[i];", "w *= d ? frac[2 - i] : 1.0 - frac[2 - i];"),
+    "weight_sign": ("w *= d ? frac[i] : 1.0 - frac[i];", "w *= d ? 1.0 - frac[i] : frac[i];"),
+    "dropped_corner": ("double w = corner(v, frac, c, vc);\n                uint32_t h = oracle_hash3(vc[0], vc[1], vc[2]) & mask;\n                for (int f = 0; f < F; ++f)\n                    acc[f]",
+                       "double w = (c == 7) ? 0.0 : corner(v, frac, c, vc);\n                uint32_t h = oracle_hash3(vc[0], vc[1], vc[2]) & mask;\n                for (int f = 0; f < F; ++f)\n                    acc[f]"),
+    "wrong_prime": ("#define ORACLE_PRIME_Z 805459861u", "#define ORACLE_PRIME_Z 805459867u"),
+    "scale_by_N_minus_1": ("float xs = xp[i] * (float)res_l;", "float xs = xp[i] * (float)(res_l - 1);"),
+    "literal_double_floor": ("if (fabs(v - r) <= 1e-9 * v)", "if (0)"),
+    "overwrite_not_add": ("dtable[((size_t)l * T + h) * F + f] +=", "dtable[((size_t)l * T + h) * F + f] ="),
+    "int64_hash_low_bits_lost": ("return (u0 * ORACLE_PRIME_X) ^ (u1 * ORACLE_PRIME_Y) ^ (u2 * ORACLE_PRIME_Z);",
+                                 "return ((u0 * ORACLE_PRIME_X) ^ (u1 * ORACLE_PRIME_Y) ^ (u2 * ORACLE_PRIME_Z)) & 0x7fffffffu;"),
+}
+
+PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+
+
+def build_mutant(tmp_path, name):
+    src = open(SRC).read()
+    old, new = MUTATIONS[name]
+    assert src.count(old) == 1, f"mutation {name} does not apply"
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / f"lib_{name}.so"
+    subprocess.run(["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
+                    "-o", str(lib), str(path), "-lm"], check=True)
+    return str(lib)
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc missing")
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_mutation(tmp_path, name, monkeypatch):
+    path = build_mutant(tmp_path, name)
+    good = oracle._lib()                      # typed prototypes of the real library
+    mut = ctypes.CDLL(path)
+    for fn in ("oracle_resolutions", "oracle_hash3", "oracle_half_to_double", "oracle_indices",
+               "oracle_forward", "oracle_backward"):
+        getattr(mut, fn).argtypes = getattr(good, fn).argtypes
+        getattr(mut, fn).restype = getattr(good, fn).restype
+    monkeypatch.setattr(oracle, "_LIB", mut)
+    failed = []
+    for t in PIN_TESTS:
+        try:
+            t()
+        except (AssertionError, ValueError):
+            failed.append(t.__name__)
+    assert failed, f"mutation {name} passed every pin"
