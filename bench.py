@@ -1,0 +1,505 @@
+#!/usr/bin/env python
+"""Benchmark of the multiresolution hash-grid encoding on B200: encoded points/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload NAME] [--skip-cpu-baseline] [--skip-e2e] [--skip-fwd-leg]
+
+One step = one pass of the whole hot path over one batch resident in HBM: zero the table
+gradient, forward (voxel, 8 corner hashes, gathers, trilinear interpolation, level-major
+output rows), backward (weighted scatter-add into the fp32 gradient table). The default
+workload is the 16-level, F=2, T=2^19 grid (N 16->512) on 2^14 rays x 64 stratified
+samples (2^20 points); the forward-only leg on 2^18 uniform points of the same grid is
+reported under "fwd". L2 is flushed (256 MiB write) before every timed step, outside the
+step's events. Rank 0 prints one JSON line.
+
+Multi-GPU: one process per GPU (torchrun); every rank encodes its own batch with its own
+table replica (points are independent), there is no collective on the data path, and the
+value is all ranks' points divided by the slowest rank's time (weak scaling).
+
+``--impl reference`` times the CPU oracle (the only reference this method has) on a
+bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from datetime import timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "encoded points/s fwd & fwd+bwd at L16 F2 T2^19; % of memory roofline"
+UNIT = "points/s"
+DEFAULT_WORKLOAD = "rays_L16F2T19"
+FWD_WORKLOAD = "grid_L16F2T19"
+FLUSH_BYTES = 256 << 20
+CPU_SAMPLE_POINTS = 1 << 18
+REFERENCE_SAMPLE_POINTS = 1 << 15
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------------------
+# Roofline arithmetic (bytes the method must move, each counted once)
+# ---------------------------------------------------------------------------------------
+
+def algorithmic_bytes_per_point(w: workloads.Workload, kind: str) -> int:
+    """fwd: 12 B of x + 8 corners x L*F table elements + 4 B per output element;
+    bwd: 12 B of x + 4 B per upstream-gradient element + 8 corners x L*F fp32 reductions."""
+    s = 2 if w.dtype == "f16" else 4
+    LF = w.L * w.F
+    fwd = 12 + 8 * LF * s + 4 * LF
+    bwd = 12 + 4 * LF + 8 * LF * 4
+    return {"fwd": fwd, "bwd": bwd, "fwdbwd": fwd + bwd}[kind]
+
+
+def measured_peaks() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def csrc_digest() -> str:
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "multiresolution_hash_grid_b200", "csrc", "*")))
+    for f in files:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str) -> float | None:
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of ``kernel`` on
+    ``workload`` from the committed ncu summary, or None when the kernel sources changed
+    since that capture."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("csrc_sha") != csrc_digest():
+        return None
+    ent = d.get("kernels", {}).get(f"{kernel}@{workload}")
+    return None if ent is None else float(ent["dram_bytes_per_launch"])
+
+
+# ---------------------------------------------------------------------------------------
+# Ranks (one process per GPU); helpers are backend-agnostic so gloo tests cover them
+# ---------------------------------------------------------------------------------------
+
+def dist_env() -> tuple[int, int, int]:
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own batch (independent units; weak scaling)."""
+    return 1000 + rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None) -> None:
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and getattr(device, "type", "cpu") == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def whole_job_rate(units_per_rank: int, world: int, max_seconds: float) -> float:
+    return units_per_rank * world / max_seconds
+
+
+# ---------------------------------------------------------------------------------------
+# Clock sampling during the timed region (NVML polling thread; nvidia-smi as fallback)
+# ---------------------------------------------------------------------------------------
+
+REASON_BITS = {  # NVML clocks-event-reason bits
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons of the current GPU while active."""
+
+    def __init__(self, device_index: int):
+        self.samples: list[tuple[float, int]] = []
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            handle = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hd = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(hd)
+                u = u.decode() if isinstance(u, bytes) else u
+                if uuid.replace("GPU-", "") in u:
+                    handle = hd
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._handle = handle
+            self._nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: the JSON line records why
+            self.error = f"nvml unavailable: {e}"
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+                self.samples.append((mhz, reasons))
+            except Exception as e:
+                self.error = str(e)
+                return
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._handle is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": self.error or "no samples"}
+        mhz = [m for m, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        reasons = sorted(n for b, n in REASON_BITS.items() if bits & b and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------------------
+# Device timing
+# ---------------------------------------------------------------------------------------
+
+class Resident:
+    """One workload's inputs and outputs resident in HBM, plus the library handle."""
+
+    def __init__(self, w: workloads.Workload, seed: int, device, backward: bool):
+        import torch
+
+        import multiresolution_hash_grid_b200 as hg
+        self.w, self.hg, self.backward = w, hg, backward
+        inp = workloads.make_inputs(w, seed=seed, grads=backward)
+        self.N = inp.x.shape[0]
+        self.x = torch.from_numpy(inp.x).to(device)
+        self.table = torch.from_numpy(inp.table).to(device)
+        self.out = torch.empty((self.N, w.L * w.F), dtype=torch.float32, device=device)
+        self.g = torch.from_numpy(inp.g).to(device) if backward else None
+        self.dtable = torch.zeros((w.L, w.T, w.F), dtype=torch.float32, device=device) if backward else None
+        dt = hg.HASHGRID_F16 if w.dtype == "f16" else hg.HASHGRID_F32
+        self.handle = hg.hashgrid_create(w.L, w.F, w.log2T, w.N_min, w.N_max, dt)
+        self.host = inp
+
+    def forward(self, stream):
+        self.hg.hashgrid_forward(self.handle, self.x, self.N, self.table, self.out, stream)
+
+    def backward_pass(self, stream):
+        self.hg.hashgrid_backward(self.handle, self.x, self.g, self.N, self.dtable, stream)
+
+    def close(self):
+        self.hg.hashgrid_destroy(self.handle)
+
+
+def time_steps(res: Resident, steps: int, warmup: int, device, sampler=None) -> dict:
+    """Times ``steps`` steps with CUDA events on the launching stream. Each step: zero the
+    gradient (if backward), forward, backward. L2 is flushed before every step, outside
+    the step's events. Returns per-phase mean milliseconds and the max-over-ranks total."""
+    import torch
+    stream = torch.cuda.current_stream(device)
+    sp = stream.cuda_stream
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def one(evs=None):
+        flush.fill_(1)
+        if evs:
+            evs[0].record(stream)
+        if res.backward:
+            res.dtable.zero_()
+        if evs:
+            evs[1].record(stream)
+        res.forward(sp)
+        if evs:
+            evs[2].record(stream)
+        if res.backward:
+            res.backward_pass(sp)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(warmup):
+        one()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    if sampler is not None:
+        sampler.__enter__()
+    for k in range(steps):
+        one(events[k])
+    torch.cuda.synchronize(device)
+    if sampler is not None:
+        sampler.__exit__(None, None, None)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    zero = [e[0].elapsed_time(e[1]) for e in events]
+    fwd = [e[1].elapsed_time(e[2]) for e in events]
+    bwd = [e[2].elapsed_time(e[3]) for e in events] if res.backward else [0.0] * steps
+    total = [e[0].elapsed_time(e[3]) for e in events]
+    total_ms = sum(total)
+    return {
+        "total_ms": total_ms,
+        "max_total_ms": max_over_ranks(total_ms, device),
+        "zero_ms": statistics.mean(zero), "fwd_ms": statistics.mean(fwd), "bwd_ms": statistics.mean(bwd),
+        "step_ms": statistics.mean(total),
+        "launches": steps * (2 if res.backward else 1),
+    }
+
+
+def time_e2e(res: Resident, steps: int, warmup: int, device) -> dict:
+    """End to end through the C ABI from pinned host buffers: per step, copy x (and the
+    upstream gradient) host->device, forward (+ zero + backward), copy the encoding back to
+    pinned host memory. The gradient table stays on the device for the optimizer."""
+    import torch
+    stream = torch.cuda.current_stream(device)
+    sp = stream.cuda_stream
+    xh = torch.from_numpy(res.host.x).pin_memory()
+    gh = torch.from_numpy(res.host.g).pin_memory() if res.backward else None
+    oh = torch.empty(res.out.shape, dtype=torch.float32).pin_memory()
+    h2d = xh.numel() * 4 + (gh.numel() * 4 if gh is not None else 0)
+    d2h = oh.numel() * 4
+
+    def one():
+        res.x.copy_(xh, non_blocking=True)
+        if gh is not None:
+            res.g.copy_(gh, non_blocking=True)
+            res.dtable.zero_()
+        res.forward(sp)
+        if res.backward:
+            res.backward_pass(sp)
+        oh.copy_(res.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(e0.elapsed_time(e1), device)
+    return {"ms": ms, "h2d": h2d, "d2h": d2h}
+
+
+def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, kernel: str) -> dict:
+    peak, src = measured_peaks()
+    bytes_per_launch = algorithmic_bytes_per_point(w, kind) * points
+    achieved = bytes_per_launch / (kernel_ms * 1e-3) / 1e9
+    traffic = ncu_traffic(kernel, w.name)
+    return {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "algorithmic_bytes_per_launch": bytes_per_launch, "kernel_ms": round(kernel_ms, 5),
+            "peak_source": f"hbm_gbs of {src} peaks"}
+
+
+def cpu_baseline(w: workloads.Workload, sample: int) -> dict:
+    import oracle
+    threads = oracle.default_threads()
+    inp = workloads.make_inputs(w, seed=rank_seed(0), n_points=sample, grads=w.backward)
+    og = oracle.Grid(w.L, w.F, w.log2T, w.N_min, w.N_max, oracle.F16 if w.dtype == "f16" else oracle.F32)
+    t0 = time.perf_counter()
+    og.forward(inp.x, inp.table, nthreads=threads)
+    if w.backward:
+        og.backward(inp.x, inp.g, nthreads=threads)
+    dt = time.perf_counter() - t0
+    n = inp.x.shape[0]
+    return {"value": round(n / dt, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"first {n} points of {w.name} (seed {rank_seed(0)}), "
+                      f"{'fwd+bwd' if w.backward else 'fwd'}; fwd parallel over points, "
+                      f"bwd over the {w.L} levels; {dt:.2f} s"}
+
+
+# ---------------------------------------------------------------------------------------
+# Arms
+# ---------------------------------------------------------------------------------------
+
+def run_reference(args) -> None:
+    """CPU oracle arm: rank 0 only (other ranks exit without work). Each step encodes a
+    bounded sample of the workload, forward and backward, on the host cores."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    w = workloads.WORKLOADS[args.workload]
+    threads = oracle.default_threads()
+    inp = workloads.make_inputs(w, seed=rank_seed(0), n_points=REFERENCE_SAMPLE_POINTS, grads=True)
+    og = oracle.Grid(w.L, w.F, w.log2T, w.N_min, w.N_max, oracle.F16 if w.dtype == "f16" else oracle.F32)
+
+    def step():
+        og.forward(inp.x, inp.table, nthreads=threads)
+        og.backward(inp.x, inp.g, nthreads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    n = inp.x.shape[0]
+    value = n * args.steps / dt
+    sample = (f"{n} points of {w.name} per step (seed {rank_seed(0)}), fwd+bwd; fwd parallel over "
+              f"points, bwd over the {w.L} levels")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "description": w.describe(),
+                                        "sample_points_per_step": n},
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_b200(args) -> None:
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    w = workloads.WORKLOADS[args.workload]
+
+    res = Resident(w, rank_seed(rank), device, backward=w.backward)
+    sampler = ClockSampler(device.index)
+    t = time_steps(res, args.steps, args.warmup, device, sampler)
+    seconds = t["max_total_ms"] * 1e-3
+    value = whole_job_rate(res.N, world, seconds)
+    launches = t["launches"]
+
+    kind, kms, kname = ("bwd", t["bwd_ms"], "backward_kernel") if t["bwd_ms"] >= t["fwd_ms"] else \
+        ("fwd", t["fwd_ms"], "forward_kernel")
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t["max_total_ms"] / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded NeRF-like ray samples; random table)",
+        "config": {"workload": w.name, "description": w.describe(), "points_per_rank": res.N,
+                   "global_points": res.N * world, "parallelism": f"dp{world}: points sharded, no collective",
+                   "step": "zero dL_dtable + forward + backward" if w.backward else "forward",
+                   "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                   "phase_ms": {"zero": round(t["zero_ms"], 5), "fwd": round(t["fwd_ms"], 5),
+                                "bwd": round(t["bwd_ms"], 5)}},
+        "roofline": roofline(w, kind, res.N, kms, kname),
+        "roofline_step": None,
+        "clocks": sampler.summary(),
+    }
+    step_bytes = algorithmic_bytes_per_point(w, "fwdbwd" if w.backward else "fwd") * res.N
+    peak, src = measured_peaks()
+    step_gbs = step_bytes / (t["step_ms"] * 1e-3) / 1e9
+    line["roofline_step"] = {"achieved": round(step_gbs, 1), "peak": peak, "unit": "GB/s",
+                             "frac": round(step_gbs / peak, 4),
+                             "note": f"whole step incl. gradient zeroing, {src} peak"}
+
+    if not args.skip_fwd_leg and w.name != FWD_WORKLOAD:
+        fw = workloads.WORKLOADS[FWD_WORKLOAD]
+        fres = Resident(fw, rank_seed(rank), device, backward=False)
+        ft = time_steps(fres, args.steps, args.warmup, device)
+        fval = whole_job_rate(fres.N, world, ft["max_total_ms"] * 1e-3)
+        line["fwd"] = {"workload": fw.name, "description": fw.describe(), "value": round(fval, 1), "unit": UNIT,
+                       "ms_per_step": round(ft["max_total_ms"] / args.steps, 5),
+                       "roofline": roofline(fw, "fwd", fres.N, ft["fwd_ms"], "forward_kernel")}
+        launches += ft["launches"]
+        fres.close()
+        del fres
+
+    if not args.skip_e2e:
+        e = time_e2e(res, args.steps, min(args.warmup, 3), device)
+        line["e2e"] = {"value": round(res.N * world * args.steps / (e["ms"] * 1e-3), 1), "unit": UNIT,
+                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                       "note": "pinned host x (and upstream grads) -> device, zero + fwd + bwd through "
+                               "the C ABI, encoding -> pinned host; the gradient table stays on the device"}
+    line["gpu_launches"] = launches
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, min(CPU_SAMPLE_POINTS, res.N))
+    res.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(device)
+        dist.destroy_process_group()
+
+
+def main(argv=None) -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-fwd-leg", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "b200":
+        print("note: fewer than 3 warm-up steps; the timing rules want at least 3", file=sys.stderr)
+    _, world, _ = dist_env()
+    if world != args.gpus:
+        print(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_b200(args)
+
+
+if __name__ == "__main__":
+    main()

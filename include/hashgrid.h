@@ -1,0 +1,161 @@
+/*
+ * hashgrid.h -- C ABI of libhashgrid.so: the multiresolution hash-grid encoding
+ * (Instant-NGP style) on NVIDIA B200 (sm_100a), forward and backward.
+ *
+ * Sources, cited by page and section:
+ *   [NeRFace-HG]  "NeRFace + Instant-NGP hash encoding" article (ipipp.com, 0929/63223),
+ *                 section 2 (二): L levels, each a table of T learnable F-wide features;
+ *                 resolution N_l growing geometrically from N_min to N_max; the point's voxel
+ *                 and its 8 corners; corner hash with primes (1, 2654435761, 805459861);
+ *                 trilinear interpolation; concatenation into an L*F vector. Section 3 (三)
+ *                 and the end of section 2: only the sampled features receive gradient.
+ *   [Repro-HG]    "Reproduce Instant-NGP's hash-encoding layer in PyTorch" (jsqmd.com,
+ *                 news/998204): section 2.1 (level table), 2.2 (XOR-of-primes hash mod T),
+ *                 3 (the layer, [B,3] -> [B,L*F]), 5 (half-precision tables; a custom CUDA
+ *                 kernel for the hash).
+ *   [Overview-HG] Instant-NGP overview (ijyty.com, news/1538821), section 2.2 (the hash
+ *                 formula; hash queries run in parallel on the GPU), section 3.1 (irregular
+ *                 table accesses are the memory bottleneck; cache hot buckets on chip).
+ *
+ * Conventions shared by every call:
+ *   - All array pointers are DEVICE pointers (cudaMalloc'd, or PyTorch CUDA tensors) on the
+ *     device that is current when the call is made, unless a parameter says otherwise.
+ *     Pointers must be 16-byte aligned; otherwise the call returns HASHGRID_ERR_ALIGN.
+ *     Pointers that the CUDA runtime does not report as device-accessible memory are
+ *     rejected with HASHGRID_ERR_ARG before anything is launched.
+ *   - Layouts (row-major, element offsets):
+ *       x          [N, 3]      fp32, x[p*3 + i]; the encoding's domain is [0,1]^3. Points
+ *                               outside are not clamped: the same formula applies (int32
+ *                               floor, uint32 hash wraparound). NaN/Inf, or |x*N_l| >= 2^31,
+ *                               give unspecified (but in-bounds) results.
+ *       table      [L, T, F]   fp32 or fp16 (the handle's dtype), table[(l*T + i)*F + f]
+ *       out        [N, L*F]    fp32, out[p*L*F + l*F + f] (level l in columns l*F..l*F+F-1)
+ *       dL_dout    [N, L*F]    fp32, same layout as out
+ *       dL_dtable  [L, T, F]   fp32 for both table dtypes
+ *   - Corner numbering: corner c in 0..7 has offsets (c & 1, (c >> 1) & 1, (c >> 2) & 1)
+ *     along (x, y, z).
+ *   - Calls are asynchronous on `cuda_stream` (a cudaStream_t; NULL = the legacy default
+ *     stream), like a kernel launch. Nothing is synchronised.
+ *   - Ownership: the caller owns every array and the stream; the library owns the handle.
+ *   - Errors: every call returns a hashgrid_status. Invalid arguments are reported before
+ *     any launch and nothing is written. A failed launch returns HASHGRID_ERR_CUDA.
+ *     hashgrid_last_error() gives a message for the last failure on the calling thread.
+ *   - N = 0 is a valid no-op (returns HASHGRID_OK, pointers may be NULL).
+ *   - A handle may be used from several threads and streams at once; it is read-only after
+ *     hashgrid_create.
+ */
+#ifndef HASHGRID_H
+#define HASHGRID_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct hashgrid_s *hashgrid_t; /* opaque, library-owned */
+
+/* Table storage type. fp16 tables are read as IEEE binary16 and converted exactly to fp32
+ * (subnormals kept); interpolation and gradients are fp32 ([Repro-HG] section 5). */
+enum hashgrid_dtype { HASHGRID_F32 = 0, HASHGRID_F16 = 1 };
+
+enum hashgrid_status {
+    HASHGRID_OK = 0,
+    HASHGRID_ERR_ARG = 1,          /* invalid argument (shape, range, NULL, host pointer) */
+    HASHGRID_ERR_ALIGN = 2,        /* a pointer is not 16-byte aligned */
+    HASHGRID_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed */
+    HASHGRID_ERR_OOM = 4,          /* host allocation of the handle failed */
+    HASHGRID_ERR_DEVICE_CHECK = 5  /* reserved: a device-side range check tripped */
+};
+
+/* Parameter limits checked by hashgrid_create. The pages use L = 16 to 32 levels
+ * ([Repro-HG] section 5, [Overview-HG] section 2.1) and F = 2 to 4 features. */
+#define HASHGRID_MAX_LEVELS 32
+#define HASHGRID_MIN_LOG2T 4
+#define HASHGRID_MAX_LOG2T 24
+#define HASHGRID_MAX_RESOLUTION (1 << 20)
+
+/*
+ * hashgrid_create -- build a handle for an encoding of L levels, F features per level,
+ * T = 2^log2T entries per level table, resolutions from N_min to N_max, table dtype.
+ *
+ * [NeRFace-HG] section 2: growth factor b = exp((ln N_max - ln N_min)/(L - 1)) and
+ * N_l = floor(N_min * b^l). The floor is taken of the exact-math value: a double result
+ * within 1e-9 (relative) of an integer is that integer (so N_{L-1} = N_max even where a
+ * literal double computation gives 4095.99999 for 4096); otherwise it is floored. L = 1
+ * requires N_min == N_max (b is undefined; N_0 = N_min).
+ *
+ * Valid ranges: 1 <= L <= 32; F in {1, 2, 4, 8}; 4 <= log2T <= 24;
+ * 1 <= N_min <= N_max <= 2^20; dtype in hashgrid_dtype. T is a power of two, so the
+ * pages' "mod T" is a mask of the hash's low bits.
+ * On success writes a new handle to *out and returns HASHGRID_OK. Does not touch the GPU.
+ */
+int hashgrid_create(int L, int F, int log2T, int N_min, int N_max, int dtype, hashgrid_t *out);
+
+/* Free a handle (NULL is allowed). The caller must not destroy a handle while calls that
+ * use it are still being issued from other threads; work already launched is unaffected. */
+int hashgrid_destroy(hashgrid_t h);
+
+/* Copy the L per-level resolutions N_l into res_out (host array of L ints). */
+int hashgrid_resolutions(hashgrid_t h, int *res_out);
+
+/* Handle parameters, for callers that allocate buffers: L*T*F, the number of elements of
+ * a table (and of dL_dtable); and L*F, the width of an output row. 0 for a NULL handle. */
+size_t hashgrid_table_elems(hashgrid_t h);
+int hashgrid_output_width(hashgrid_t h);
+
+/* The create arguments of a handle, written to the non-NULL pointers (host ints). */
+int hashgrid_params(hashgrid_t h, int *L, int *F, int *log2T, int *N_min, int *N_max, int *dtype);
+
+/*
+ * hashgrid_forward -- encode N points.
+ *
+ * [NeRFace-HG] section 2, [Repro-HG] section 3: for each point p and level l,
+ *   xs = fp32(x * N_l) per axis, v = floor(xs), frac = xs - v;
+ *   corner c = v + offsets(c); index_c = hash(corner_c) mod T, with
+ *   hash(c) = c0*1 XOR c1*2654435761 XOR c2*805459861 in uint32 wraparound
+ *   ([Repro-HG] section 2.2, [Overview-HG] section 2.2);
+ *   w_c = prod over axes of (frac_i if offset_i else 1 - frac_i);
+ *   out[p][l*F + f] = sum_c w_c * table[l][index_c][f]   (fp32 arithmetic).
+ *
+ * x: [N,3] fp32; table: [L,T,F] of the handle's dtype; out: [N,L*F] fp32 (overwritten).
+ */
+int hashgrid_forward(hashgrid_t h, const float *x, int64_t N, const void *table, float *out,
+                     void *cuda_stream);
+
+/*
+ * hashgrid_backward -- gradient of a loss with respect to the tables.
+ *
+ * The forward pass is linear in the table, and only the entries a point's corners read
+ * receive gradient ([NeRFace-HG] end of section 2 and section 3):
+ *   dL_dtable[l][index_c][f] += w_c * dL_dout[p][l*F + f]   for every p, l, c.
+ * dL_dtable is ACCUMULATED into (fp32 atomic reductions; the caller zeroes it first when
+ * a fresh gradient is wanted). Colliding corners each add their own contribution. The
+ * summation order is unspecified, so results vary in the last bits from run to run.
+ *
+ * x: [N,3] fp32; dL_dout: [N,L*F] fp32; dL_dtable: [L,T,F] fp32 (for both table dtypes).
+ */
+int hashgrid_backward(hashgrid_t h, const float *x, const float *dL_dout, int64_t N,
+                      float *dL_dtable, void *cuda_stream);
+
+/*
+ * hashgrid_debug_indices -- export the hash index of every corner: idx_out[(p*L + l)*8 + c]
+ * = index_c of point p at level l (uint32, < T), computed by the same device code as the
+ * forward and backward passes. For tests and inspection. idx_out: [N, L, 8] uint32.
+ */
+int hashgrid_debug_indices(hashgrid_t h, const float *x, int64_t N, uint32_t *idx_out,
+                           void *cuda_stream);
+
+/* Message describing the last failed call on the calling thread ("" if none). The pointer
+ * stays valid until the next call on this thread. */
+const char *hashgrid_last_error(void);
+
+/* Library version string. */
+const char *hashgrid_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HASHGRID_H */

@@ -1,0 +1,178 @@
+"""Python binding of libhashgrid.so, the B200 (sm_100a) multiresolution hash-grid encoding.
+
+Argument marshalling only: every step of the encoding runs in the library's CUDA kernels.
+PyTorch supplies device memory and streams. The functions carry the C ABI's names
+(``include/hashgrid.h`` documents semantics, layouts and errors) and take either torch
+CUDA tensors or raw integer device pointers; ``stream`` defaults to torch's current
+stream. A nonzero status raises ``HashGridError`` with the library's message.
+
+The library must be built (``python multiresolution_hash_grid_b200/build.py``); importing
+this package without it raises ImportError. There is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libhashgrid.so")
+
+HASHGRID_F32 = 0
+HASHGRID_F16 = 1
+
+HASHGRID_OK = 0
+HASHGRID_ERR_ARG = 1
+HASHGRID_ERR_ALIGN = 2
+HASHGRID_ERR_CUDA = 3
+HASHGRID_ERR_OOM = 4
+HASHGRID_ERR_DEVICE_CHECK = 5
+
+MAX_LEVELS = 32
+
+
+class HashGridError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"hashgrid error {code}: {message}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built: run `python multiresolution_hash_grid_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    i32, i64, vp, sz = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+    protos = {
+        "hashgrid_create": (i32, [i32, i32, i32, i32, i32, i32, ctypes.POINTER(vp)]),
+        "hashgrid_destroy": (i32, [vp]),
+        "hashgrid_resolutions": (i32, [vp, ctypes.POINTER(i32)]),
+        "hashgrid_table_elems": (sz, [vp]),
+        "hashgrid_output_width": (i32, [vp]),
+        "hashgrid_params": (i32, [vp] + [ctypes.POINTER(i32)] * 6),
+        "hashgrid_forward": (i32, [vp, vp, i64, vp, vp, vp]),
+        "hashgrid_backward": (i32, [vp, vp, vp, i64, vp, vp]),
+        "hashgrid_debug_indices": (i32, [vp, vp, i64, vp, vp]),
+        "hashgrid_last_error": (ctypes.c_char_p, []),
+        "hashgrid_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in protos.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    return lib
+
+
+lib = _load()
+
+
+def _check(rc: int) -> None:
+    if rc != HASHGRID_OK:
+        raise HashGridError(rc, lib.hashgrid_last_error().decode())
+
+
+def _ptr(a) -> int | None:
+    if a is None:
+        return None
+    if isinstance(a, int):
+        return a
+    return a.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def hashgrid_version() -> str:
+    return lib.hashgrid_version().decode()
+
+
+def hashgrid_last_error() -> str:
+    return lib.hashgrid_last_error().decode()
+
+
+def hashgrid_create(L: int, F: int, log2T: int, N_min: int, N_max: int, dtype: int = HASHGRID_F32) -> int:
+    h = ctypes.c_void_p()
+    _check(lib.hashgrid_create(L, F, log2T, N_min, N_max, dtype, ctypes.byref(h)))
+    return h.value
+
+
+def hashgrid_destroy(h: int) -> None:
+    _check(lib.hashgrid_destroy(h))
+
+
+def hashgrid_params(h: int) -> dict:
+    vals = [ctypes.c_int() for _ in range(6)]
+    _check(lib.hashgrid_params(h, *[ctypes.byref(v) for v in vals]))
+    return dict(zip(("L", "F", "log2T", "N_min", "N_max", "dtype"), (v.value for v in vals)))
+
+
+def hashgrid_resolutions(h: int) -> list[int]:
+    arr = (ctypes.c_int * MAX_LEVELS)()
+    _check(lib.hashgrid_resolutions(h, arr))
+    return list(arr[: hashgrid_params(h)["L"]])
+
+
+def hashgrid_table_elems(h: int) -> int:
+    return int(lib.hashgrid_table_elems(h))
+
+
+def hashgrid_output_width(h: int) -> int:
+    return int(lib.hashgrid_output_width(h))
+
+
+def hashgrid_forward(h: int, x, N: int, table, out, stream=None) -> None:
+    _check(lib.hashgrid_forward(h, _ptr(x), N, _ptr(table), _ptr(out), _stream(stream)))
+
+
+def hashgrid_backward(h: int, x, dL_dout, N: int, dL_dtable, stream=None) -> None:
+    _check(lib.hashgrid_backward(h, _ptr(x), _ptr(dL_dout), N, _ptr(dL_dtable), _stream(stream)))
+
+
+def hashgrid_debug_indices(h: int, x, N: int, idx_out, stream=None) -> None:
+    _check(lib.hashgrid_debug_indices(h, _ptr(x), N, _ptr(idx_out), _stream(stream)))
+
+
+class HashGrid:
+    """Owns a handle and allocates outputs with torch; the encoding itself runs in the
+    library. ``table`` arguments are CUDA tensors of shape [L, T, F] (float32 or float16,
+    matching ``dtype``)."""
+
+    def __init__(self, L: int = 16, F: int = 2, log2T: int = 19, N_min: int = 16, N_max: int = 512,
+                 dtype: int = HASHGRID_F32):
+        self.L, self.F, self.log2T, self.N_min, self.N_max, self.dtype = L, F, log2T, N_min, N_max, dtype
+        self.T = 1 << log2T
+        self.handle = hashgrid_create(L, F, log2T, N_min, N_max, dtype)
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            lib.hashgrid_destroy(h)
+            self.handle = None
+
+    @property
+    def resolutions(self) -> list[int]:
+        return hashgrid_resolutions(self.handle)
+
+    def forward(self, x, table, out=None, stream=None):
+        import torch
+        N = x.shape[0]
+        if out is None:
+            out = torch.empty((N, self.L * self.F), dtype=torch.float32, device=x.device)
+        hashgrid_forward(self.handle, x, N, table, out, stream)
+        return out
+
+    def backward(self, x, dL_dout, dL_dtable=None, stream=None):
+        import torch
+        if dL_dtable is None:
+            dL_dtable = torch.zeros((self.L, self.T, self.F), dtype=torch.float32, device=x.device)
+        hashgrid_backward(self.handle, x, dL_dout, x.shape[0], dL_dtable, stream)
+        return dL_dtable
+
+    def indices(self, x, stream=None):
+        import torch
+        idx = torch.empty((x.shape[0], self.L, 8), dtype=torch.int32, device=x.device)
+        hashgrid_debug_indices(self.handle, x, x.shape[0], idx, stream)
+        return idx

@@ -1,0 +1,312 @@
+// hashgrid.cu -- C ABI of libhashgrid.so (declared in include/hashgrid.h): handle, host-side
+// validation and kernel launches for the multiresolution hash-grid encoding on sm_100a.
+//
+// Every argument is checked on the host before anything is launched: ranges, NULLs,
+// 16-byte alignment, that each pointer is device-accessible memory of the current device,
+// and (for cudaMalloc'd memory) that the whole extent the call will touch lies inside the
+// pointer's allocation. A call either launches its kernels or returns an error having
+// written nothing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "hashgrid.h"
+#include "hg_device.cuh"
+
+#define HASHGRID_VERSION_STRING "hashgrid-b200 0.1 (sm_100a)"
+
+struct hashgrid_s {
+    int L, F, log2T, N_min, N_max, dtype;
+    int res[HASHGRID_MAX_LEVELS];
+    hg::LevelParams lp;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int ok() { return HASHGRID_OK; }
+
+// Resolution schedule, [NeRFace-HG] section 2: b = exp((ln N_max - ln N_min)/(L - 1)),
+// N_l = floor(N_min * b^l) of the exact-math value. In double, N_min * b^l can fall a few
+// ulp short of an integer it equals exactly (16 * b^15 = 4095.99999... for N_max = 4096);
+// a value within 1e-9 (relative) of an integer is taken as that integer, any other value
+// is floored.
+bool compute_resolutions(int L, int N_min, int N_max, int* res) {
+    if (L == 1) {
+        if (N_min != N_max) return false;
+        res[0] = N_min;
+        return true;
+    }
+    const double b = std::exp((std::log((double)N_max) - std::log((double)N_min)) / (double)(L - 1));
+    for (int l = 0; l < L; ++l) {
+        const double v = (double)N_min * std::pow(b, (double)l);
+        const double r = std::nearbyint(v);
+        res[l] = (int)((std::fabs(v - r) <= 1e-9 * v) ? r : std::floor(v));
+    }
+    return true;
+}
+
+// cuMemGetAddressRange through the runtime's driver entry-point query, so the library
+// needs no link-time dependency on libcuda.
+typedef CUresult (*PFN_memGetAddressRange)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+PFN_memGetAddressRange address_range_fn() {
+    static PFN_memGetAddressRange fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            p = nullptr;
+        }
+        return reinterpret_cast<PFN_memGetAddressRange>(p);
+    }();
+    return fn;
+}
+
+// Checks one buffer argument that the call will access over [p, p + bytes).
+int check_buffer(const void* p, size_t bytes, const char* name) {
+    if (p == nullptr) return fail(HASHGRID_ERR_ARG, "%s is NULL", name);
+    if (reinterpret_cast<uintptr_t>(p) % 16 != 0)
+        return fail(HASHGRID_ERR_ALIGN, "%s (%p) is not 16-byte aligned", name, p);
+    cudaPointerAttributes a;
+    cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(HASHGRID_ERR_ARG, "%s (%p): cudaPointerGetAttributes failed: %s", name, p,
+                    cudaGetErrorString(e));
+    }
+    if (a.type == cudaMemoryTypeUnregistered || a.devicePointer == nullptr)
+        return fail(HASHGRID_ERR_ARG, "%s (%p) is not device-accessible memory", name, p);
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(HASHGRID_ERR_CUDA, "cudaGetDevice failed");
+    }
+    if (a.type == cudaMemoryTypeDevice) {
+        if (a.device != dev)
+            return fail(HASHGRID_ERR_ARG, "%s lives on device %d but device %d is current", name,
+                        a.device, dev);
+        PFN_memGetAddressRange range = address_range_fn();
+        if (range != nullptr) {
+            CUdeviceptr base = 0;
+            size_t size = 0;
+            if (range(&base, &size, (CUdeviceptr)(uintptr_t)p) == CUDA_SUCCESS) {
+                const uintptr_t end = (uintptr_t)base + size;
+                if ((uintptr_t)p + bytes > end || (uintptr_t)p + bytes < (uintptr_t)p)
+                    return fail(HASHGRID_ERR_ARG,
+                                "%s: the call touches %zu bytes from %p but its allocation ends "
+                                "%zu bytes after it",
+                                name, bytes, p, (size_t)(end - (uintptr_t)p));
+            }
+        }
+    }
+    return ok();
+}
+
+int check_handle(const hashgrid_s* h) {
+    if (h == nullptr) return fail(HASHGRID_ERR_ARG, "handle is NULL");
+    return ok();
+}
+
+int check_N(int64_t N, int BP) {
+    if (N < 0) return fail(HASHGRID_ERR_ARG, "N = %lld is negative", (long long)N);
+    if ((N + BP - 1) / BP > 0x7fffffffLL)
+        return fail(HASHGRID_ERR_ARG, "N = %lld exceeds the largest launchable batch", (long long)N);
+    return ok();
+}
+
+int launch_status(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(HASHGRID_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+    return ok();
+}
+
+constexpr int kTile = 64;      // points per block tile
+constexpr int kMaxThreads = 512;
+
+int tile_threads(int L) {
+    const int items = (kTile / 32) * L;
+    return items * 32 < kMaxThreads ? items * 32 : kMaxThreads;
+}
+
+template <typename K>
+int prepare_smem(K kernel, size_t smem) {
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return fail(HASHGRID_ERR_CUDA, "cudaFuncSetAttribute(smem=%zu) failed: %s", smem,
+                        cudaGetErrorString(e));
+        }
+    }
+    return ok();
+}
+
+template <int F, typename TT>
+int launch_forward(const hashgrid_s* h, const float* x, int64_t N, const void* table, float* out,
+                   cudaStream_t s) {
+    auto k = hg::forward_kernel<F, TT, kTile>;
+    const size_t smem = hg::tile_smem_bytes(kTile, h->L, F);
+    if (int rc = prepare_smem(k, smem)) return rc;
+    const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
+    k<<<blocks, tile_threads(h->L), smem, s>>>(h->lp, x, N, static_cast<const TT*>(table), out);
+    return launch_status("forward");
+}
+
+template <int F>
+int launch_backward(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
+                    float* dtable, cudaStream_t s) {
+    auto k = hg::backward_kernel<F, kTile>;
+    const size_t smem = hg::tile_smem_bytes(kTile, h->L, F);
+    if (int rc = prepare_smem(k, smem)) return rc;
+    const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
+    k<<<blocks, tile_threads(h->L), smem, s>>>(h->lp, x, dout, N, dtable);
+    return launch_status("backward");
+}
+
+size_t table_bytes(const hashgrid_s* h) {
+    return (size_t)h->L * ((size_t)1 << h->log2T) * (size_t)h->F * (h->dtype == HASHGRID_F16 ? 2 : 4);
+}
+
+}  // namespace
+
+extern "C" {
+
+int hashgrid_create(int L, int F, int log2T, int N_min, int N_max, int dtype, hashgrid_t* out) {
+    if (out == nullptr) return fail(HASHGRID_ERR_ARG, "out handle pointer is NULL");
+    *out = nullptr;
+    if (L < 1 || L > HASHGRID_MAX_LEVELS)
+        return fail(HASHGRID_ERR_ARG, "L = %d outside [1, %d]", L, HASHGRID_MAX_LEVELS);
+    if (F != 1 && F != 2 && F != 4 && F != 8)
+        return fail(HASHGRID_ERR_ARG, "F = %d not in {1, 2, 4, 8}", F);
+    if (log2T < HASHGRID_MIN_LOG2T || log2T > HASHGRID_MAX_LOG2T)
+        return fail(HASHGRID_ERR_ARG, "log2T = %d outside [%d, %d]", log2T, HASHGRID_MIN_LOG2T,
+                    HASHGRID_MAX_LOG2T);
+    if (N_min < 1 || N_max < N_min || N_max > HASHGRID_MAX_RESOLUTION)
+        return fail(HASHGRID_ERR_ARG, "resolutions N_min = %d, N_max = %d outside 1 <= N_min <= N_max <= %d",
+                    N_min, N_max, HASHGRID_MAX_RESOLUTION);
+    if (dtype != HASHGRID_F32 && dtype != HASHGRID_F16)
+        return fail(HASHGRID_ERR_ARG, "dtype = %d is neither HASHGRID_F32 nor HASHGRID_F16", dtype);
+    if (L == 1 && N_min != N_max)
+        return fail(HASHGRID_ERR_ARG, "L = 1 needs N_min == N_max (the growth factor divides by L - 1)");
+    hashgrid_s* h = new (std::nothrow) hashgrid_s;
+    if (h == nullptr) return fail(HASHGRID_ERR_OOM, "out of host memory");
+    std::memset(h, 0, sizeof(*h));
+    h->L = L; h->F = F; h->log2T = log2T; h->N_min = N_min; h->N_max = N_max; h->dtype = dtype;
+    compute_resolutions(L, N_min, N_max, h->res);
+    h->lp.L = L;
+    h->lp.T = (uint64_t)1 << log2T;
+    h->lp.mask = (uint32_t)(h->lp.T - 1);
+    for (int l = 0; l < L; ++l) h->lp.scale[l] = (float)h->res[l];
+    *out = h;
+    return ok();
+}
+
+int hashgrid_destroy(hashgrid_t h) {
+    delete h;
+    return ok();
+}
+
+int hashgrid_resolutions(hashgrid_t h, int* res_out) {
+    if (int rc = check_handle(h)) return rc;
+    if (res_out == nullptr) return fail(HASHGRID_ERR_ARG, "res_out is NULL");
+    std::memcpy(res_out, h->res, sizeof(int) * h->L);
+    return ok();
+}
+
+size_t hashgrid_table_elems(hashgrid_t h) {
+    if (h == nullptr) return 0;
+    return (size_t)h->L * ((size_t)1 << h->log2T) * (size_t)h->F;
+}
+
+int hashgrid_output_width(hashgrid_t h) { return h == nullptr ? 0 : h->L * h->F; }
+
+int hashgrid_params(hashgrid_t h, int* L, int* F, int* log2T, int* N_min, int* N_max, int* dtype) {
+    if (int rc = check_handle(h)) return rc;
+    if (L) *L = h->L;
+    if (F) *F = h->F;
+    if (log2T) *log2T = h->log2T;
+    if (N_min) *N_min = h->N_min;
+    if (N_max) *N_max = h->N_max;
+    if (dtype) *dtype = h->dtype;
+    return ok();
+}
+
+int hashgrid_forward(hashgrid_t h, const float* x, int64_t N, const void* table, float* out,
+                     void* cuda_stream) {
+    if (int rc = check_handle(h)) return rc;
+    if (int rc = check_N(N, kTile)) return rc;
+    if (N == 0) return ok();
+    const size_t W = (size_t)h->L * h->F;
+    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(table, table_bytes(h), "table")) return rc;
+    if (int rc = check_buffer(out, (size_t)N * W * sizeof(float), "out")) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    const bool half = h->dtype == HASHGRID_F16;
+    switch (h->F) {
+        case 1: return half ? launch_forward<1, __half>(h, x, N, table, out, s) : launch_forward<1, float>(h, x, N, table, out, s);
+        case 2: return half ? launch_forward<2, __half>(h, x, N, table, out, s) : launch_forward<2, float>(h, x, N, table, out, s);
+        case 4: return half ? launch_forward<4, __half>(h, x, N, table, out, s) : launch_forward<4, float>(h, x, N, table, out, s);
+        case 8: return half ? launch_forward<8, __half>(h, x, N, table, out, s) : launch_forward<8, float>(h, x, N, table, out, s);
+    }
+    return fail(HASHGRID_ERR_ARG, "corrupt handle");
+}
+
+int hashgrid_backward(hashgrid_t h, const float* x, const float* dL_dout, int64_t N, float* dL_dtable,
+                      void* cuda_stream) {
+    if (int rc = check_handle(h)) return rc;
+    if (int rc = check_N(N, kTile)) return rc;
+    if (N == 0) return ok();
+    const size_t W = (size_t)h->L * h->F;
+    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(dL_dout, (size_t)N * W * sizeof(float), "dL_dout")) return rc;
+    if (int rc = check_buffer(dL_dtable, hashgrid_table_elems(h) * sizeof(float), "dL_dtable")) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    switch (h->F) {
+        case 1: return launch_backward<1>(h, x, dL_dout, N, dL_dtable, s);
+        case 2: return launch_backward<2>(h, x, dL_dout, N, dL_dtable, s);
+        case 4: return launch_backward<4>(h, x, dL_dout, N, dL_dtable, s);
+        case 8: return launch_backward<8>(h, x, dL_dout, N, dL_dtable, s);
+    }
+    return fail(HASHGRID_ERR_ARG, "corrupt handle");
+}
+
+int hashgrid_debug_indices(hashgrid_t h, const float* x, int64_t N, uint32_t* idx_out, void* cuda_stream) {
+    if (int rc = check_handle(h)) return rc;
+    if (int rc = check_N(N, 1)) return rc;
+    if (N == 0) return ok();
+    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(idx_out, (size_t)N * h->L * 8 * sizeof(uint32_t), "idx_out")) return rc;
+    const int64_t total = N * h->L;
+    const int threads = 256;
+    const int64_t blocks = (total + threads - 1) / threads;
+    if (blocks > 0x7fffffffLL) return fail(HASHGRID_ERR_ARG, "N too large for the index export");
+    hg::indices_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+        h->lp, x, N, idx_out);
+    return launch_status("debug_indices");
+}
+
+const char* hashgrid_last_error(void) { return g_last_error.c_str(); }
+
+const char* hashgrid_version(void) { return HASHGRID_VERSION_STRING; }
+
+}  // extern "C"

@@ -1,0 +1,364 @@
+// hg_device.cuh -- device code of the multiresolution hash-grid encoding for sm_100a.
+//
+// Sources (cited by page and section; see include/hashgrid.h for the full list):
+//   [NeRFace-HG] section 2: voxel of the scaled point, 8 corners, corner hash, trilinear
+//                interpolation, concatenation of levels; end of section 2 and section 3:
+//                only the sampled table entries receive gradient.
+//   [Repro-HG]   section 2.2 (hash), section 3 (layer), section 5 (fp16 tables, a CUDA
+//                kernel for the hash).
+//   [Overview-HG] section 2.2 (hash formula), section 3.1 (table reads are irregular; the
+//                cache hierarchy is what limits them).
+//
+// Work decomposition. One thread computes one (point, level) pair. A warp always holds 32
+// consecutive points of a block tile at ONE level, so its 8 corner gathers per lane hit
+// one level's table and neighbouring points share cache sectors. A block owns a tile of BP
+// points: it stages the tile's x rows (and, in the backward pass, the upstream-gradient
+// rows) in shared memory with coalesced loads, runs its warps over the tile's
+// (32-point group, level) items, and (forward) writes the [BP, L*F] output tile back with
+// contiguous vector stores. Nothing is saved between forward and backward; the backward
+// pass recomputes voxel, indices and weights.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace hg {
+
+constexpr int kMaxLevels = 32;
+constexpr uint32_t kPrimeY = 2654435761u;  // [NeRFace-HG] section 2; [Repro-HG] section 2.2
+constexpr uint32_t kPrimeZ = 805459861u;   // (the x prime is 1)
+
+// Per-call level parameters, passed by value (kernel parameter space, read with uniform
+// indices by each warp).
+struct LevelParams {
+    float scale[kMaxLevels];  // (float)N_l
+    uint32_t mask;            // T - 1
+    int L;
+    uint64_t T;               // entries per level table
+};
+
+// Shared-memory row stride (in floats) of a staged [BP, L*F] tile. The padding keeps the
+// per-lane row writes of one level conflict-free for F-wide vector stores.
+__host__ __device__ constexpr int row_pad(int F) { return F < 4 ? F : 4; }
+
+// ---------------------------------------------------------------------------------------
+// Table entry loads (read-only path). F fp32 or fp16 values -> F fp32 registers.
+// fp16 -> fp32 conversion is exact (binary16 values, subnormals included, are all
+// representable in binary32).
+// ---------------------------------------------------------------------------------------
+template <int F, typename TT> struct EntryLoad;
+
+template <> struct EntryLoad<1, float> {
+    static __device__ __forceinline__ void load(const float* p, float* e) { e[0] = __ldg(p); }
+};
+template <> struct EntryLoad<2, float> {
+    static __device__ __forceinline__ void load(const float* p, float* e) {
+        float2 v = __ldg(reinterpret_cast<const float2*>(p));
+        e[0] = v.x; e[1] = v.y;
+    }
+};
+template <> struct EntryLoad<4, float> {
+    static __device__ __forceinline__ void load(const float* p, float* e) {
+        float4 v = __ldg(reinterpret_cast<const float4*>(p));
+        e[0] = v.x; e[1] = v.y; e[2] = v.z; e[3] = v.w;
+    }
+};
+template <> struct EntryLoad<8, float> {
+    static __device__ __forceinline__ void load(const float* p, float* e) {
+        float4 a = __ldg(reinterpret_cast<const float4*>(p));
+        float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+        e[0] = a.x; e[1] = a.y; e[2] = a.z; e[3] = a.w;
+        e[4] = b.x; e[5] = b.y; e[6] = b.z; e[7] = b.w;
+    }
+};
+template <> struct EntryLoad<1, __half> {
+    static __device__ __forceinline__ void load(const __half* p, float* e) {
+        e[0] = __half2float(__ldg(p));
+    }
+};
+template <> struct EntryLoad<2, __half> {
+    static __device__ __forceinline__ void load(const __half* p, float* e) {
+        float2 v = __half22float2(__ldg(reinterpret_cast<const __half2*>(p)));
+        e[0] = v.x; e[1] = v.y;
+    }
+};
+__device__ __forceinline__ float2 h2_bits_to_f2(uint32_t bits) {
+    __half2 h = *reinterpret_cast<__half2*>(&bits);
+    return __half22float2(h);
+}
+template <> struct EntryLoad<4, __half> {
+    static __device__ __forceinline__ void load(const __half* p, float* e) {
+        uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+        float2 a = h2_bits_to_f2(v.x), b = h2_bits_to_f2(v.y);
+        e[0] = a.x; e[1] = a.y; e[2] = b.x; e[3] = b.y;
+    }
+};
+template <> struct EntryLoad<8, __half> {
+    static __device__ __forceinline__ void load(const __half* p, float* e) {
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+        float2 a = h2_bits_to_f2(v.x), b = h2_bits_to_f2(v.y);
+        float2 c = h2_bits_to_f2(v.z), d = h2_bits_to_f2(v.w);
+        e[0] = a.x; e[1] = a.y; e[2] = b.x; e[3] = b.y;
+        e[4] = c.x; e[5] = c.y; e[6] = d.x; e[7] = d.y;
+    }
+};
+
+// ---------------------------------------------------------------------------------------
+// fp32 vector reductions into global memory (red.global.add, vector forms are sm_90+).
+// ---------------------------------------------------------------------------------------
+template <int F> struct RedAdd;
+template <> struct RedAdd<1> {
+    static __device__ __forceinline__ void add(float* p, const float* v) {
+        asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v[0]) : "memory");
+    }
+};
+template <> struct RedAdd<2> {
+    static __device__ __forceinline__ void add(float* p, const float* v) {
+        asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(v[0]), "f"(v[1])
+                     : "memory");
+    }
+};
+template <> struct RedAdd<4> {
+    static __device__ __forceinline__ void add(float* p, const float* v) {
+        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v[0]),
+                     "f"(v[1]), "f"(v[2]), "f"(v[3])
+                     : "memory");
+    }
+};
+template <> struct RedAdd<8> {
+    static __device__ __forceinline__ void add(float* p, const float* v) {
+        RedAdd<4>::add(p, v);
+        RedAdd<4>::add(p + 4, v + 4);
+    }
+};
+
+// ---------------------------------------------------------------------------------------
+// Voxel, corner indices and trilinear weights of one point at one level.
+// [NeRFace-HG] section 2: xs = x * N_l (one fp32 multiply, never fused), v = floor(xs),
+// frac = xs - v (exact in fp32). The hash of corner v + d is
+//   (v0 + d0) XOR (v1 + d1) * P_y XOR (v2 + d2) * P_z   (mod 2^32),
+// and (v_i + 1) * P = v_i * P + P mod 2^32, so each axis needs one multiply for both of
+// its offsets. Weight of corner c: product over axes of frac_i (offset 1) or 1 - frac_i.
+// ---------------------------------------------------------------------------------------
+struct Corners {
+    uint32_t idx[8];
+    float w[8];
+};
+
+__device__ __forceinline__ void locate_corners(float x0, float x1, float x2, float scale,
+                                               uint32_t mask, Corners& cr) {
+    const float xs0 = __fmul_rn(x0, scale);
+    const float xs1 = __fmul_rn(x1, scale);
+    const float xs2 = __fmul_rn(x2, scale);
+    const int v0 = __float2int_rd(xs0);
+    const int v1 = __float2int_rd(xs1);
+    const int v2 = __float2int_rd(xs2);
+    const float f0 = __fsub_rn(xs0, __int2float_rn(v0));
+    const float f1 = __fsub_rn(xs1, __int2float_rn(v1));
+    const float f2 = __fsub_rn(xs2, __int2float_rn(v2));
+    const uint32_t hx0 = (uint32_t)v0, hx1 = hx0 + 1u;
+    const uint32_t hy0 = (uint32_t)v1 * kPrimeY, hy1 = hy0 + kPrimeY;
+    const uint32_t hz0 = (uint32_t)v2 * kPrimeZ, hz1 = hz0 + kPrimeZ;
+    const float g0 = 1.0f - f0, g1 = 1.0f - f1, g2 = 1.0f - f2;
+    const float wxy[4] = {g0 * g1, f0 * g1, g0 * f1, f0 * f1};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint32_t hx = (c & 1) ? hx1 : hx0;
+        const uint32_t hy = (c & 2) ? hy1 : hy0;
+        const uint32_t hz = (c & 4) ? hz1 : hz0;
+        cr.idx[c] = (hx ^ hy ^ hz) & mask;
+        cr.w[c] = wxy[c & 3] * ((c & 4) ? f2 : g2);
+    }
+}
+
+// Stage rows [p0, p0 + nvalid) of a global [*, W] fp32 array into shared memory with row
+// stride S (coalesced global reads, V-wide).
+template <int V>
+__device__ __forceinline__ void stage_rows_in(float* s, const float* __restrict__ gsrc,
+                                              int64_t p0, int nvalid, int W, int S) {
+    const int per_row = W / V;
+    const int total = nvalid * per_row;
+    const float* base = gsrc + p0 * (int64_t)W;
+    for (int k = threadIdx.x; k < total; k += blockDim.x) {
+        const int row = k / per_row;
+        const int col = (k - row * per_row) * V;
+        if constexpr (V == 4) {
+            float4 v = __ldcs(reinterpret_cast<const float4*>(base + (int64_t)row * W + col));
+            *reinterpret_cast<float4*>(s + row * S + col) = v;
+        } else if constexpr (V == 2) {
+            float2 v = __ldcs(reinterpret_cast<const float2*>(base + (int64_t)row * W + col));
+            *reinterpret_cast<float2*>(s + row * S + col) = v;
+        } else {
+            s[row * S + col] = __ldcs(base + (int64_t)row * W + col);
+        }
+    }
+}
+
+template <int V>
+__device__ __forceinline__ void stage_rows_out(const float* s, float* __restrict__ gdst,
+                                               int64_t p0, int nvalid, int W, int S) {
+    const int per_row = W / V;
+    const int total = nvalid * per_row;
+    float* base = gdst + p0 * (int64_t)W;
+    for (int k = threadIdx.x; k < total; k += blockDim.x) {
+        const int row = k / per_row;
+        const int col = (k - row * per_row) * V;
+        if constexpr (V == 4) {
+            __stcs(reinterpret_cast<float4*>(base + (int64_t)row * W + col),
+                   *reinterpret_cast<const float4*>(s + row * S + col));
+        } else if constexpr (V == 2) {
+            __stcs(reinterpret_cast<float2*>(base + (int64_t)row * W + col),
+                   *reinterpret_cast<const float2*>(s + row * S + col));
+        } else {
+            __stcs(base + (int64_t)row * W + col, s[row * S + col]);
+        }
+    }
+}
+
+template <int F>
+__device__ __forceinline__ void store_smem_entry(float* s, const float* v) {
+    if constexpr (F == 1) {
+        s[0] = v[0];
+    } else if constexpr (F == 2) {
+        *reinterpret_cast<float2*>(s) = make_float2(v[0], v[1]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < F; j += 4)
+            *reinterpret_cast<float4*>(s + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+}
+
+template <int F>
+__device__ __forceinline__ void load_smem_entry(const float* s, float* v) {
+    if constexpr (F == 1) {
+        v[0] = s[0];
+    } else if constexpr (F == 2) {
+        float2 a = *reinterpret_cast<const float2*>(s);
+        v[0] = a.x; v[1] = a.y;
+    } else {
+#pragma unroll
+        for (int j = 0; j < F; j += 4) {
+            float4 a = *reinterpret_cast<const float4*>(s + j);
+            v[j] = a.x; v[j + 1] = a.y; v[j + 2] = a.z; v[j + 3] = a.w;
+        }
+    }
+}
+
+// Dynamic shared memory of one block: x tile [BP*3] then a data tile [BP * S].
+__host__ __device__ constexpr size_t tile_smem_bytes(int BP, int L, int F) {
+    return sizeof(float) * ((size_t)BP * 3 + (size_t)BP * (L * F + row_pad(F)));
+}
+
+// ---------------------------------------------------------------------------------------
+// Forward kernel. Grid: one block per BP-point tile.
+// ---------------------------------------------------------------------------------------
+template <int F, typename TT, int BP>
+__global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const float* __restrict__ x,
+                                                      int64_t N, const TT* __restrict__ table,
+                                                      float* __restrict__ out) {
+    extern __shared__ __align__(16) float smem[];
+    const int L = lp.L;
+    const int W = L * F;
+    const int S = W + row_pad(F);
+    float* xs = smem;
+    float* os = smem + BP * 3;
+    const int64_t p0 = (int64_t)blockIdx.x * BP;
+    const int nvalid = (int)min((int64_t)BP, N - p0);
+
+    for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = __ldcs(x + p0 * 3 + i);
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const int items = (BP / 32) * L;
+#pragma unroll 2
+    for (int it = warp; it < items; it += nwarps) {
+        const int q = it / L;
+        const int l = it - q * L;
+        const int pl = q * 32 + lane;
+        if (pl < nvalid) {
+            Corners cr;
+            locate_corners(xs[pl * 3 + 0], xs[pl * 3 + 1], xs[pl * 3 + 2], lp.scale[l], lp.mask, cr);
+            const TT* tl = table + (uint64_t)l * lp.T * F;
+            float e[8][F];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) EntryLoad<F, TT>::load(tl + (uint64_t)cr.idx[c] * F, e[c]);
+            float o[F];
+#pragma unroll
+            for (int f = 0; f < F; ++f) {
+                float acc = cr.w[0] * e[0][f];
+#pragma unroll
+                for (int c = 1; c < 8; ++c) acc = fmaf(cr.w[c], e[c][f], acc);
+                o[f] = acc;
+            }
+            store_smem_entry<F>(os + pl * S + l * F, o);
+        }
+    }
+    __syncthreads();
+    stage_rows_out<(F < 4 ? F : 4)>(os, out, p0, nvalid, W, S);
+}
+
+// ---------------------------------------------------------------------------------------
+// Backward kernel (table gradient). Grid: one block per BP-point tile. Each (point, level,
+// corner) issues one F-wide fp32 reduction of w_c * dL_dout[p][l*F..] into the level's
+// gradient table.
+// ---------------------------------------------------------------------------------------
+template <int F, int BP>
+__global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const float* __restrict__ x,
+                                                       const float* __restrict__ dout, int64_t N,
+                                                       float* __restrict__ dtable) {
+    extern __shared__ __align__(16) float smem[];
+    const int L = lp.L;
+    const int W = L * F;
+    const int S = W + row_pad(F);
+    float* xs = smem;
+    float* gs = smem + BP * 3;
+    const int64_t p0 = (int64_t)blockIdx.x * BP;
+    const int nvalid = (int)min((int64_t)BP, N - p0);
+
+    for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = __ldcs(x + p0 * 3 + i);
+    stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const int items = (BP / 32) * L;
+    for (int it = warp; it < items; it += nwarps) {
+        const int q = it / L;
+        const int l = it - q * L;
+        const int pl = q * 32 + lane;
+        if (pl < nvalid) {
+            Corners cr;
+            locate_corners(xs[pl * 3 + 0], xs[pl * 3 + 1], xs[pl * 3 + 2], lp.scale[l], lp.mask, cr);
+            float g[F];
+            load_smem_entry<F>(gs + pl * S + l * F, g);
+            float* dl = dtable + (uint64_t)l * lp.T * F;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float v[F];
+#pragma unroll
+                for (int f = 0; f < F; ++f) v[f] = cr.w[c] * g[f];
+                RedAdd<F>::add(dl + (uint64_t)cr.idx[c] * F, v);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Index export (tests and inspection): idx[(p*L + l)*8 + c]. One thread per (point, level).
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) indices_kernel(LevelParams lp, const float* __restrict__ x,
+                                                      int64_t N, uint32_t* __restrict__ idx) {
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t total = N * lp.L;
+    if (t >= total) return;
+    const int64_t p = t / lp.L;
+    const int l = (int)(t - p * lp.L);
+    Corners cr;
+    locate_corners(x[p * 3 + 0], x[p * 3 + 1], x[p * 3 + 2], lp.scale[l], lp.mask, cr);
+    uint4* dst = reinterpret_cast<uint4*>(idx + t * 8);
+    dst[0] = make_uint4(cr.idx[0], cr.idx[1], cr.idx[2], cr.idx[3]);
+    dst[1] = make_uint4(cr.idx[4], cr.idx[5], cr.idx[6], cr.idx[7]);
+}
+
+}  // namespace hg

@@ -1,0 +1,292 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle.
+
+Bars (from the method's arithmetic, see the design notes):
+  - hash indices: bit-exact;
+  - forward: |gpu - ref| <= rtol * sum_c w_c |e_c| + 1e-30 per element, with rtol 1e-6 for
+    fp32 tables and 2e-3 for fp16 tables. sum_c w_c |e_c| is the oracle's encoding of the
+    absolute-value table; an error bound relative to it stays meaningful when features
+    cancel to near zero, where a plain relative error is ill-conditioned;
+  - backward: ||g - g_ref||_2 / ||g_ref||_2 <= 1e-5 over the gradient table (fp32 atomics
+    accumulate in an unspecified order).
+Reduced sizes span many 64-point tiles plus a ragged tail; full sizes run the library's
+own launch configuration (the one the benchmark times) and compare sampled rows, level
+subsets of the gradient, and the adjoint identity, which holds at any size.
+"""
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+FWD_RTOL = {"f32": 1e-6, "f16": 2e-3}
+BWD_REL_L2 = 1e-5
+THREADS = oracle.default_threads()
+
+
+def hgmod():
+    import multiresolution_hash_grid_b200 as hg
+    return hg
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def make_pair(L, F, log2T, N_min, N_max, dtype="f32"):
+    hg = hgmod()
+    dt = hg.HASHGRID_F16 if dtype == "f16" else hg.HASHGRID_F32
+    return hg.HashGrid(L, F, log2T, N_min, N_max, dt), oracle.Grid(L, F, log2T, N_min, N_max,
+                                                                    oracle.F16 if dtype == "f16" else oracle.F32)
+
+
+def gpu_forward(grid, x, table):
+    out = grid.forward(dev(x), dev(table))
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def gpu_backward(grid, x, g):
+    d = grid.backward(dev(x), dev(g))
+    torch.cuda.synchronize()
+    return d.cpu().numpy()
+
+
+def abs_table(table):
+    return np.abs(table)
+
+
+def check_forward(og, x, table, got, dtype, rows=None):
+    ref = og.forward(x, table, nthreads=THREADS)
+    bound = og.forward(x, abs_table(table), nthreads=THREADS)
+    if rows is not None:
+        got = got[rows]
+    err = np.abs(got.astype(np.float64) - ref)
+    lim = FWD_RTOL[dtype] * bound + 1e-30
+    bad = np.argwhere(err > lim)
+    assert bad.size == 0, f"{len(bad)} elements off; first {bad[:5].tolist()} err {err[tuple(bad[0])]:.3e} lim {lim[tuple(bad[0])]:.3e}"
+    return ref
+
+
+def rel_l2(got, ref):
+    ref = ref.astype(np.float64)
+    den = np.linalg.norm(ref.ravel())
+    return np.linalg.norm(got.astype(np.float64).ravel() - ref.ravel()) / max(den, 1e-300)
+
+
+# ---------------------------------------------------------------------------------------
+# The five workloads at reduced sizes (several tiles + a ragged tail)
+# ---------------------------------------------------------------------------------------
+
+REDUCED_N = 4096 + 37
+
+
+@pytest.fixture(scope="module")
+def reduced_inputs():
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            w = workloads.WORKLOADS[name]
+            n = w.n_points if w.n_points <= 4096 else REDUCED_N
+            cache[name] = (w, workloads.make_inputs(w, seed=0, n_points=n, grads=True))
+        return cache[name]
+    return get
+
+
+@pytest.mark.parametrize("name", list(workloads.WORKLOADS))
+def test_indices_bit_exact(name, reduced_inputs):
+    w, inp = reduced_inputs(name)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype)
+    got = grid.indices(dev(inp.x)).cpu().numpy().view(np.uint32)
+    want = og.indices(inp.x)
+    np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("name", list(workloads.WORKLOADS))
+def test_forward_parity(name, reduced_inputs):
+    w, inp = reduced_inputs(name)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype)
+    got = gpu_forward(grid, inp.x, inp.table)
+    check_forward(og, inp.x, inp.table, got, w.dtype)
+
+
+@pytest.mark.parametrize("name", list(workloads.WORKLOADS))
+def test_backward_parity(name, reduced_inputs):
+    w, inp = reduced_inputs(name)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype)
+    got = gpu_backward(grid, inp.x, inp.g)
+    ref = og.backward(inp.x, inp.g, nthreads=THREADS)
+    assert rel_l2(got, ref) <= BWD_REL_L2
+    # untouched entries stay exactly zero; touched ones are nonzero on both sides
+    np.testing.assert_array_equal(got == 0, ref == 0)
+
+
+# ---------------------------------------------------------------------------------------
+# Full sizes, in the launch configuration the benchmark times
+# ---------------------------------------------------------------------------------------
+
+FULL_LEVELS = {   # gradient levels the oracle recomputes at full size (bounded CPU time)
+    "tiny_L4F2T10": [(0, 4)],
+    "rays_L16F2T19": [(0, 16)],
+    "half_L16F2T19": [(0, 1), (8, 9), (15, 16)],
+    "large_L16F4T22": [(0, 1), (15, 16)],
+}
+
+
+@pytest.mark.parametrize("name", list(workloads.WORKLOADS))
+def test_full_size(name):
+    w = workloads.WORKLOADS[name]
+    inp = workloads.make_inputs(w, seed=0, grads=True)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype)
+    x_d, t_d, g_d = dev(inp.x), dev(inp.table), dev(inp.g)
+    out_d = grid.forward(x_d, t_d)
+    dt_d = grid.backward(x_d, g_d)
+    torch.cuda.synchronize()
+    # forward: sampled rows (random, first and last tiles)
+    N = inp.x.shape[0]
+    rng = np.random.default_rng(99)
+    rows = np.unique(np.concatenate([rng.choice(N, 2048, replace=False), np.arange(64), np.arange(N - 64, N)]))
+    got_rows = out_d[torch.from_numpy(rows).cuda()].cpu().numpy()
+    check_forward(og, inp.x[rows], inp.table, got_rows, w.dtype)
+    # adjoint identity <g, fwd(t)> == <bwd(g), t>, computed in fp64 on the device
+    tf = t_d.double()
+    lhs = float(torch.sum(g_d.double() * out_d.double()))
+    rhs = float(torch.sum(dt_d.double() * tf))
+    assert abs(lhs - rhs) <= 1e-5 * max(abs(lhs), abs(rhs), 1e-30)
+    # gradient: level subsets against the oracle
+    if name in FULL_LEVELS:
+        got = dt_d.cpu().numpy()
+        for l0, l1 in FULL_LEVELS[name]:
+            ref = np.zeros((w.L, w.T, w.F))
+            og.backward(inp.x, inp.g, levels=(l0, l1), nthreads=THREADS, dtable=ref)
+            assert rel_l2(got[l0:l1], ref[l0:l1]) <= BWD_REL_L2, (l0, l1)
+
+
+# ---------------------------------------------------------------------------------------
+# Edge cases
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N", [1, 2, 31, 32, 33, 63, 64, 65, 127, 129, 1000])
+def test_ragged_batch_sizes(N):
+    grid, og = make_pair(16, 2, 19, 16, 512)
+    rng = np.random.default_rng(N)
+    table = workloads.table_values(rng, 16, 2**19, 2)
+    x = workloads.uniform_points(rng, N)
+    g = workloads.upstream_grads(rng, N, 32)
+    check_forward(og, x, table, gpu_forward(grid, x, table), "f32")
+    assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g, nthreads=THREADS)) <= BWD_REL_L2
+
+
+def test_special_coordinates():
+    """x = 0, the largest fp32 below 1, exactly 1 (voxel N_l, corner N_l + 1), points
+    outside the cube (no clamping), and grid vertices (bit-exact table entries)."""
+    grid, og = make_pair(4, 2, 10, 2, 16)
+    rng = np.random.default_rng(5)
+    table = rng.standard_normal((4, 1024, 2)).astype(np.float32)
+    vals = np.array([0.0, 1.0 - 2**-24, 1.0, 0.5, 0.25, -0.3, 1.7, -2.0, 3.25], dtype=np.float32)
+    x = np.stack(np.meshgrid(vals, vals, vals, indexing="ij"), -1).reshape(-1, 3).astype(np.float32)
+    got = gpu_forward(grid, x, table)
+    check_forward(og, x, table, got, "f32")
+    np.testing.assert_array_equal(grid.indices(dev(x)).cpu().numpy().view(np.uint32), og.indices(x))
+    # vertices: x = k/2 lands on a vertex at every level of the 2->16 grid
+    k = rng.integers(0, 3, size=(200, 3))
+    xv = (k / 2.0).astype(np.float32)
+    np.testing.assert_array_equal(gpu_forward(grid, xv, table), og.forward(xv, table).astype(np.float32))
+    g = rng.standard_normal((x.shape[0], 8)).astype(np.float32)
+    assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g)) <= BWD_REL_L2
+
+
+@pytest.mark.parametrize("F", [1, 2, 4, 8])
+@pytest.mark.parametrize("dtype", ["f32", "f16"])
+def test_feature_widths_and_dtypes(F, dtype):
+    grid, og = make_pair(5, F, 12, 3, 200, dtype)
+    rng = np.random.default_rng(F)
+    table = workloads.table_values(rng, 5, 2**12, F, dtype)
+    x = workloads.uniform_points(rng, 3000)
+    g = workloads.upstream_grads(rng, 3000, 5 * F)
+    check_forward(og, x, table, gpu_forward(grid, x, table), dtype)
+    assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g, nthreads=THREADS)) <= BWD_REL_L2
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 2, 10, 64, 64),          # L = 1, N_min == N_max
+    (32, 2, 14, 16, 2**20),      # most levels, largest resolution
+    (3, 2, 4, 4, 64),            # T = 16: corners of one point collide
+    (2, 1, 24, 512, 2**16),      # largest table
+    (32, 8, 8, 2, 300),          # widest output row (256 floats, > 48 KB of shared memory)
+])
+def test_extreme_shapes(shape):
+    L, F, log2T, a, b = shape
+    grid, og = make_pair(L, F, log2T, a, b)
+    rng = np.random.default_rng(L * 100 + F)
+    table = workloads.table_values(rng, L, 2**log2T, F)
+    x = workloads.uniform_points(rng, 777)
+    g = workloads.upstream_grads(rng, 777, L * F)
+    np.testing.assert_array_equal(grid.indices(dev(x)).cpu().numpy().view(np.uint32), og.indices(x))
+    check_forward(og, x, table, gpu_forward(grid, x, table), "f32")
+    assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g, nthreads=THREADS)) <= BWD_REL_L2
+
+
+def test_backward_accumulates_and_side_stream():
+    grid, og = make_pair(16, 2, 19, 16, 512)
+    w = workloads.WORKLOADS["rays_L16F2T19"]
+    inp = workloads.make_inputs(w, seed=3, n_points=2000)
+    s = torch.cuda.Stream()
+    x_d, g_d = dev(inp.x), dev(inp.g)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        d = torch.zeros((16, 2**19, 2), device="cuda")
+        grid.backward(x_d, g_d, d)
+        grid.backward(x_d, g_d, d)
+        out = grid.forward(x_d, dev(inp.table))
+    s.synchronize()
+    ref = og.backward(inp.x, inp.g, nthreads=THREADS)
+    assert rel_l2(d.cpu().numpy(), 2 * ref) <= BWD_REL_L2
+    check_forward(og, inp.x, inp.table, out.cpu().numpy(), "f32")
+
+
+def test_errors_on_device():
+    hg = hgmod()
+    grid = hg.HashGrid(4, 2, 10, 2, 16)
+    x = torch.rand(100, 3, device="cuda")
+    t = torch.zeros(4, 1024, 2, device="cuda")
+    out = torch.full((100, 8), 7.0, device="cuda")
+    L = hg.lib
+    # host memory
+    xh = np.zeros((100, 3), dtype=np.float32)
+    assert L.hashgrid_forward(grid.handle, xh.ctypes.data, 100, t.data_ptr(), out.data_ptr(), None) == hg.HASHGRID_ERR_ARG
+    # misaligned device pointer
+    assert L.hashgrid_forward(grid.handle, x.data_ptr() + 4, 99, t.data_ptr(), out.data_ptr(), None) == hg.HASHGRID_ERR_ALIGN
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)
+
+
+def test_allocation_too_small_is_rejected():
+    """With torch's caching allocator off every tensor is its own cudaMalloc, so the
+    library's allocation-range check must reject a batch larger than x's allocation. The
+    case is sized so that, were the check missing, the over-read would stay inside the
+    allocation's page (no fault); the assertion on the status would then fail."""
+    code = r"""
+import torch, numpy as np, multiresolution_hash_grid_b200 as hg
+g = hg.HashGrid(4, 2, 10, 2, 16)
+x = torch.rand(1000, 3, device="cuda")
+t = torch.zeros(4, 1024, 2, device="cuda")
+out = torch.full((2000, 8), 7.0, device="cuda")
+rc = hg.lib.hashgrid_forward(g.handle, x.data_ptr(), 2000, t.data_ptr(), out.data_ptr(), None)
+torch.cuda.synchronize()
+assert rc == hg.HASHGRID_ERR_ARG, rc
+assert "allocation" in hg.hashgrid_last_error()
+assert bool(torch.all(out == 7.0))
+print("ok")
+"""
+    env = dict(os.environ, PYTORCH_NO_CUDA_MEMORY_CACHING="1")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
