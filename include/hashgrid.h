@@ -151,6 +151,39 @@ int hashgrid_debug_indices(hashgrid_t h, const float *x, int64_t N, uint32_t *id
  * stays valid until the next call on this thread. */
 const char *hashgrid_last_error(void);
 
+/*
+ * Execution options of a handle (defaults: AUTO). Options only select among kernels that
+ * compute the same result; set them before issuing calls with the handle (they are not
+ * synchronised with calls running on other threads).
+ *
+ * HASHGRID_OPT_FORWARD_GATHER -- how the forward pass reads table entries:
+ *   HASHGRID_GATHER_CORNER: one F-wide load per corner;
+ *   HASHGRID_GATHER_SECTOR: one 256-bit load of the aligned 32-byte sector holding corner
+ *     (v0, y, z), which often also holds corner (v0 + 1, y, z) because the x prime is 1
+ *     ([NeRFace-HG] section 2: primes (1, 2654435761, 805459861)); the second corner is
+ *     loaded separately only when it is not in that sector. Needs a 32-byte-aligned table
+ *     (HASHGRID_ERR_ALIGN otherwise);
+ *   HASHGRID_GATHER_AUTO: SECTOR when the table is 32-byte aligned, else CORNER.
+ * HASHGRID_OPT_BACKWARD_MODE -- how the backward pass reduces into dL_dtable:
+ *   HASHGRID_BACKWARD_ATOMIC: each (point, level) reduces its 8 corner contributions, the
+ *     two x-corners merged into one 16-byte reduction when they share an aligned unit;
+ *   HASHGRID_BACKWARD_WARP_DEDUP: each warp (32 consecutive points at one level) first sums
+ *     its contributions per distinct 16-byte gradient unit in shared memory, then issues one
+ *     reduction per unit. Pays off for coherent batches (consecutive samples along rays)
+ *     where neighbouring points share corners. Needs F <= 4;
+ *   HASHGRID_BACKWARD_AUTO: ATOMIC.
+ * Returns HASHGRID_ERR_ARG for an unknown option or value.
+ */
+enum hashgrid_option { HASHGRID_OPT_FORWARD_GATHER = 0, HASHGRID_OPT_BACKWARD_MODE = 1 };
+enum hashgrid_gather { HASHGRID_GATHER_AUTO = 0, HASHGRID_GATHER_CORNER = 1, HASHGRID_GATHER_SECTOR = 2 };
+enum hashgrid_backward_mode {
+    HASHGRID_BACKWARD_AUTO = 0,
+    HASHGRID_BACKWARD_ATOMIC = 1,
+    HASHGRID_BACKWARD_WARP_DEDUP = 2
+};
+int hashgrid_set_option(hashgrid_t h, int option, int value);
+int hashgrid_get_option(hashgrid_t h, int option, int *value);
+
 /* Library version string. */
 const char *hashgrid_version(void);
 

@@ -29,6 +29,15 @@ HASHGRID_ERR_DEVICE_CHECK = 5
 
 MAX_LEVELS = 32
 
+HASHGRID_OPT_FORWARD_GATHER = 0
+HASHGRID_OPT_BACKWARD_MODE = 1
+HASHGRID_GATHER_AUTO = 0
+HASHGRID_GATHER_CORNER = 1
+HASHGRID_GATHER_SECTOR = 2
+HASHGRID_BACKWARD_AUTO = 0
+HASHGRID_BACKWARD_ATOMIC = 1
+HASHGRID_BACKWARD_WARP_DEDUP = 2
+
 
 class HashGridError(RuntimeError):
     def __init__(self, code: int, message: str):
@@ -48,6 +57,8 @@ def _load() -> ctypes.CDLL:
         "hashgrid_table_elems": (sz, [vp]),
         "hashgrid_output_width": (i32, [vp]),
         "hashgrid_params": (i32, [vp] + [ctypes.POINTER(i32)] * 6),
+        "hashgrid_set_option": (i32, [vp, i32, i32]),
+        "hashgrid_get_option": (i32, [vp, i32, ctypes.POINTER(i32)]),
         "hashgrid_forward": (i32, [vp, vp, i64, vp, vp, vp]),
         "hashgrid_backward": (i32, [vp, vp, vp, i64, vp, vp]),
         "hashgrid_debug_indices": (i32, [vp, vp, i64, vp, vp]),
@@ -115,6 +126,16 @@ def hashgrid_resolutions(h: int) -> list[int]:
     return list(arr[: hashgrid_params(h)["L"]])
 
 
+def hashgrid_set_option(h: int, option: int, value: int) -> None:
+    _check(lib.hashgrid_set_option(h, option, value))
+
+
+def hashgrid_get_option(h: int, option: int) -> int:
+    v = ctypes.c_int()
+    _check(lib.hashgrid_get_option(h, option, ctypes.byref(v)))
+    return v.value
+
+
 def hashgrid_table_elems(h: int) -> int:
     return int(lib.hashgrid_table_elems(h))
 
@@ -141,10 +162,13 @@ class HashGrid:
     matching ``dtype``)."""
 
     def __init__(self, L: int = 16, F: int = 2, log2T: int = 19, N_min: int = 16, N_max: int = 512,
-                 dtype: int = HASHGRID_F32):
+                 dtype: int = HASHGRID_F32, forward_gather: int = HASHGRID_GATHER_AUTO,
+                 backward_mode: int = HASHGRID_BACKWARD_AUTO):
         self.L, self.F, self.log2T, self.N_min, self.N_max, self.dtype = L, F, log2T, N_min, N_max, dtype
         self.T = 1 << log2T
         self.handle = hashgrid_create(L, F, log2T, N_min, N_max, dtype)
+        hashgrid_set_option(self.handle, HASHGRID_OPT_FORWARD_GATHER, forward_gather)
+        hashgrid_set_option(self.handle, HASHGRID_OPT_BACKWARD_MODE, backward_mode)
 
     def __del__(self):
         h = getattr(self, "handle", None)

@@ -24,6 +24,8 @@
 struct hashgrid_s {
     int L, F, log2T, N_min, N_max, dtype;
     int res[HASHGRID_MAX_LEVELS];
+    int forward_gather;   // HASHGRID_GATHER_*
+    int backward_mode;    // HASHGRID_BACKWARD_*
     hg::LevelParams lp;
 };
 
@@ -163,8 +165,8 @@ int prepare_smem(K kernel, size_t smem) {
 
 template <int F, typename TT>
 int launch_forward(const hashgrid_s* h, const float* x, int64_t N, const void* table, float* out,
-                   cudaStream_t s) {
-    auto k = hg::forward_kernel<F, TT, kTile>;
+                   bool sector, cudaStream_t s) {
+    auto k = sector ? hg::forward_kernel<F, TT, kTile, true> : hg::forward_kernel<F, TT, kTile, false>;
     const size_t smem = hg::tile_smem_bytes(kTile, h->L, F);
     if (int rc = prepare_smem(k, smem)) return rc;
     const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
@@ -172,15 +174,26 @@ int launch_forward(const hashgrid_s* h, const float* x, int64_t N, const void* t
     return launch_status("forward");
 }
 
+template <int F, bool kDedup>
+int launch_backward_mode(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
+                         float* dtable, cudaStream_t s) {
+    auto k = hg::backward_kernel<F, kTile, kDedup>;
+    const int threads = tile_threads(h->L);
+    const size_t smem = hg::tile_smem_bytes(kTile, h->L, F) + (kDedup ? hg::dedup_smem_bytes(threads / 32) : 0);
+    if (int rc = prepare_smem(k, smem)) return rc;
+    const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
+    k<<<blocks, threads, smem, s>>>(h->lp, x, dout, N, dtable);
+    return launch_status("backward");
+}
+
 template <int F>
 int launch_backward(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
                     float* dtable, cudaStream_t s) {
-    auto k = hg::backward_kernel<F, kTile>;
-    const size_t smem = hg::tile_smem_bytes(kTile, h->L, F);
-    if (int rc = prepare_smem(k, smem)) return rc;
-    const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
-    k<<<blocks, tile_threads(h->L), smem, s>>>(h->lp, x, dout, N, dtable);
-    return launch_status("backward");
+    if constexpr (F <= 4) {
+        if (h->backward_mode == HASHGRID_BACKWARD_WARP_DEDUP)
+            return launch_backward_mode<F, true>(h, x, dout, N, dtable, s);
+    }
+    return launch_backward_mode<F, false>(h, x, dout, N, dtable, s);
 }
 
 size_t table_bytes(const hashgrid_s* h) {
@@ -240,6 +253,35 @@ size_t hashgrid_table_elems(hashgrid_t h) {
 
 int hashgrid_output_width(hashgrid_t h) { return h == nullptr ? 0 : h->L * h->F; }
 
+int hashgrid_set_option(hashgrid_t h, int option, int value) {
+    if (int rc = check_handle(h)) return rc;
+    switch (option) {
+        case HASHGRID_OPT_FORWARD_GATHER:
+            if (value < HASHGRID_GATHER_AUTO || value > HASHGRID_GATHER_SECTOR)
+                return fail(HASHGRID_ERR_ARG, "forward gather mode %d is not a HASHGRID_GATHER_* value", value);
+            h->forward_gather = value;
+            return ok();
+        case HASHGRID_OPT_BACKWARD_MODE:
+            if (value < HASHGRID_BACKWARD_AUTO || value > HASHGRID_BACKWARD_WARP_DEDUP)
+                return fail(HASHGRID_ERR_ARG, "backward mode %d is not a HASHGRID_BACKWARD_* value", value);
+            if (value == HASHGRID_BACKWARD_WARP_DEDUP && h->F > 4)
+                return fail(HASHGRID_ERR_ARG, "warp dedup needs F <= 4 (16-byte gradient units), F = %d", h->F);
+            h->backward_mode = value;
+            return ok();
+    }
+    return fail(HASHGRID_ERR_ARG, "unknown option %d", option);
+}
+
+int hashgrid_get_option(hashgrid_t h, int option, int* value) {
+    if (int rc = check_handle(h)) return rc;
+    if (value == nullptr) return fail(HASHGRID_ERR_ARG, "value is NULL");
+    switch (option) {
+        case HASHGRID_OPT_FORWARD_GATHER: *value = h->forward_gather; return ok();
+        case HASHGRID_OPT_BACKWARD_MODE: *value = h->backward_mode; return ok();
+    }
+    return fail(HASHGRID_ERR_ARG, "unknown option %d", option);
+}
+
 int hashgrid_params(hashgrid_t h, int* L, int* F, int* log2T, int* N_min, int* N_max, int* dtype) {
     if (int rc = check_handle(h)) return rc;
     if (L) *L = h->L;
@@ -262,11 +304,16 @@ int hashgrid_forward(hashgrid_t h, const float* x, int64_t N, const void* table,
     if (int rc = check_buffer(out, (size_t)N * W * sizeof(float), "out")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     const bool half = h->dtype == HASHGRID_F16;
+    // Sector gathers issue 256-bit loads, which need a 32-byte-aligned table.
+    const bool aligned32 = reinterpret_cast<uintptr_t>(table) % 32 == 0;
+    bool sector = h->forward_gather != HASHGRID_GATHER_CORNER && aligned32;
+    if (h->forward_gather == HASHGRID_GATHER_SECTOR && !aligned32)
+        return fail(HASHGRID_ERR_ALIGN, "sector gathers need a 32-byte-aligned table (%p)", table);
     switch (h->F) {
-        case 1: return half ? launch_forward<1, __half>(h, x, N, table, out, s) : launch_forward<1, float>(h, x, N, table, out, s);
-        case 2: return half ? launch_forward<2, __half>(h, x, N, table, out, s) : launch_forward<2, float>(h, x, N, table, out, s);
-        case 4: return half ? launch_forward<4, __half>(h, x, N, table, out, s) : launch_forward<4, float>(h, x, N, table, out, s);
-        case 8: return half ? launch_forward<8, __half>(h, x, N, table, out, s) : launch_forward<8, float>(h, x, N, table, out, s);
+        case 1: return half ? launch_forward<1, __half>(h, x, N, table, out, sector, s) : launch_forward<1, float>(h, x, N, table, out, sector, s);
+        case 2: return half ? launch_forward<2, __half>(h, x, N, table, out, sector, s) : launch_forward<2, float>(h, x, N, table, out, sector, s);
+        case 4: return half ? launch_forward<4, __half>(h, x, N, table, out, sector, s) : launch_forward<4, float>(h, x, N, table, out, sector, s);
+        case 8: return half ? launch_forward<8, __half>(h, x, N, table, out, sector, s) : launch_forward<8, float>(h, x, N, table, out, sector, s);
     }
     return fail(HASHGRID_ERR_ARG, "corrupt handle");
 }

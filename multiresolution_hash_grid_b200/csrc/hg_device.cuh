@@ -104,6 +104,60 @@ template <> struct EntryLoad<8, __half> {
 };
 
 // ---------------------------------------------------------------------------------------
+// Sector gathers. The x prime is 1, so the two corners that differ only in x, v0 and
+// v0 + 1, hash to (v0 ^ K) and ((v0 + 1) ^ K) for the same K = hash of (y, z): their
+// indices agree in every bit above the lowest carry of v0 + 1. Whenever both land in the
+// same aligned 32-byte sector of the table, one 256-bit load (sm_100) fetches both entries
+// and the L1 sends one sector request to L2 instead of two. The second corner is loaded
+// separately only when it lies in another sector.
+// ---------------------------------------------------------------------------------------
+template <int F, typename TT>
+struct Sector {
+    static constexpr int kEntryBytes = F * (int)sizeof(TT);       // 2 .. 32
+    static constexpr int kPerSector = 32 / kEntryBytes;            // entries per sector
+    static constexpr int kWords = kEntryBytes >= 4 ? kEntryBytes / 4 : 1;  // words per entry
+};
+
+__device__ __forceinline__ void ld_sector(const void* p, uint32_t (&w)[8]) {
+    asm("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
+          "=r"(w[7])
+        : "l"(p));
+}
+
+// Entry j (0 <= j < kPerSector) of a loaded sector as F fp32 values (select chains, no
+// local-memory indexing).
+template <int F, typename TT>
+__device__ __forceinline__ void sector_entry(const uint32_t (&w)[8], uint32_t j, float* e) {
+    using S = Sector<F, TT>;
+    constexpr int WE = S::kWords;
+    constexpr int G = 8 / WE;                // word groups in a sector
+    uint32_t sel[WE];
+    const uint32_t jw = (S::kEntryBytes >= 4) ? j : (j >> 1);
+#pragma unroll
+    for (int k = 0; k < WE; ++k) {
+        uint32_t v = w[k];
+#pragma unroll
+        for (int g = 1; g < G; ++g) v = (jw == (uint32_t)g) ? w[g * WE + k] : v;
+        sel[k] = v;
+    }
+    if constexpr (sizeof(TT) == 4) {
+#pragma unroll
+        for (int f = 0; f < F; ++f) e[f] = __uint_as_float(sel[f]);
+    } else if constexpr (S::kEntryBytes >= 4) {
+#pragma unroll
+        for (int k = 0; k < WE; ++k) {
+            float2 v = h2_bits_to_f2(sel[k]);
+            e[2 * k] = v.x;
+            e[2 * k + 1] = v.y;
+        }
+    } else {  // one fp16 value: low or high half of the selected word
+        const uint32_t bits = (j & 1) ? (sel[0] >> 16) : (sel[0] & 0xffffu);
+        e[0] = __half2float(__ushort_as_half((unsigned short)bits));
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // fp32 vector reductions into global memory (red.global.add, vector forms are sm_90+).
 // ---------------------------------------------------------------------------------------
 template <int F> struct RedAdd;
@@ -131,6 +185,34 @@ template <> struct RedAdd<8> {
         RedAdd<4>::add(p + 4, v + 4);
     }
 };
+
+// Reduction of the x-corner pair (a, b) of one (y, z) edge: when both entries fall in the
+// same aligned 16-byte unit of the gradient table (F <= 2), one red.v4 carries both (the
+// unit's other elements receive +0.0, which leaves them unchanged); otherwise two F-wide
+// reductions are issued.
+template <int F>
+__device__ __forceinline__ void red_pair(float* dl, uint32_t a, uint32_t b, const float* va,
+                                         const float* vb) {
+    if constexpr (F <= 2) {
+        constexpr uint32_t kUnit = 4 / F;  // entries per 16-byte unit
+        if ((a ^ b) < kUnit) {
+            float u[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint32_t oa = (a & (kUnit - 1)) * F, ob = (b & (kUnit - 1)) * F;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                for (int f = 0; f < F; ++f) {
+                    if (oa + f == (uint32_t)k) u[k] += va[f];
+                    if (ob + f == (uint32_t)k) u[k] += vb[f];
+                }
+            }
+            RedAdd<4>::add(dl + (uint64_t)(a & ~(kUnit - 1)) * F, u);
+            return;
+        }
+    }
+    RedAdd<F>::add(dl + (uint64_t)a * F, va);
+    RedAdd<F>::add(dl + (uint64_t)b * F, vb);
+}
 
 // ---------------------------------------------------------------------------------------
 // Voxel, corner indices and trilinear weights of one point at one level.
@@ -251,8 +333,41 @@ __host__ __device__ constexpr size_t tile_smem_bytes(int BP, int L, int F) {
 
 // ---------------------------------------------------------------------------------------
 // Forward kernel. Grid: one block per BP-point tile.
+// kSector = false: one F-wide load per corner. kSector = true: one 256-bit sector load per
+// x-corner pair plus a predicated load of the second corner when it lies in another
+// sector (needs a 32-byte-aligned table).
 // ---------------------------------------------------------------------------------------
-template <int F, typename TT, int BP>
+template <int F, typename TT, bool kSector>
+__device__ __forceinline__ void gather_corners(const TT* __restrict__ tl, const Corners& cr,
+                                               float (&e)[8][F]) {
+    if constexpr (!kSector) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) EntryLoad<F, TT>::load(tl + (uint64_t)cr.idx[c] * F, e[c]);
+    } else {
+        using S = Sector<F, TT>;
+        constexpr uint32_t kPer = S::kPerSector;
+        uint32_t w[4][8];
+        float far[4][F];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t a = cr.idx[2 * q], b = cr.idx[2 * q + 1];
+            ld_sector(tl + (uint64_t)(a & ~(kPer - 1)) * F, w[q]);
+            if ((a ^ b) >= kPer) EntryLoad<F, TT>::load(tl + (uint64_t)b * F, far[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t a = cr.idx[2 * q], b = cr.idx[2 * q + 1];
+            sector_entry<F, TT>(w[q], a & (kPer - 1), e[2 * q]);
+            float near[F];
+            sector_entry<F, TT>(w[q], b & (kPer - 1), near);
+            const bool same = (a ^ b) < kPer;
+#pragma unroll
+            for (int f = 0; f < F; ++f) e[2 * q + 1][f] = same ? near[f] : far[q][f];
+        }
+    }
+}
+
+template <int F, typename TT, int BP, bool kSector>
 __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const float* __restrict__ x,
                                                       int64_t N, const TT* __restrict__ table,
                                                       float* __restrict__ out) {
@@ -271,7 +386,6 @@ __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const floa
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
     const int items = (BP / 32) * L;
-#pragma unroll 2
     for (int it = warp; it < items; it += nwarps) {
         const int q = it / L;
         const int l = it - q * L;
@@ -281,8 +395,7 @@ __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const floa
             locate_corners(xs[pl * 3 + 0], xs[pl * 3 + 1], xs[pl * 3 + 2], lp.scale[l], lp.mask, cr);
             const TT* tl = table + (uint64_t)l * lp.T * F;
             float e[8][F];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) EntryLoad<F, TT>::load(tl + (uint64_t)cr.idx[c] * F, e[c]);
+            gather_corners<F, TT, kSector>(tl, cr, e);
             float o[F];
 #pragma unroll
             for (int f = 0; f < F; ++f) {
@@ -299,14 +412,45 @@ __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const floa
 }
 
 // ---------------------------------------------------------------------------------------
-// Backward kernel (table gradient). Grid: one block per BP-point tile. Each (point, level,
-// corner) issues one F-wide fp32 reduction of w_c * dL_dout[p][l*F..] into the level's
-// gradient table.
+// Backward kernel (table gradient). Grid: one block per BP-point tile.
+//
+// kDedup = false: each lane reduces its own 8 contributions w_c * g into the level's
+// gradient table, the two x-corners of an edge merged into one 16-byte red when they share
+// an aligned unit (red_pair).
+//
+// kDedup = true (coherent batches, e.g. consecutive samples along rays): a warp first sums
+// its 32 x 8 contributions per 16-byte gradient unit in a shared-memory open-addressing
+// table (keys = unit index within the level, 256 slots, values = 4 fp32), then issues one
+// red.v4 per distinct unit. Consecutive samples of a ray share voxels at coarse levels and
+// voxel faces at finer ones, so far fewer reductions reach L2.
 // ---------------------------------------------------------------------------------------
-template <int F, int BP>
+constexpr int kDedupSlots = 256;
+constexpr uint32_t kEmptyKey = 0xffffffffu;
+
+__host__ __device__ constexpr size_t dedup_smem_bytes(int warps) {
+    return (size_t)warps * kDedupSlots * (sizeof(uint32_t) + 4 * sizeof(float));
+}
+
+template <int F>
+__device__ __forceinline__ void dedup_add(uint32_t* keys, float* vals, uint32_t idx, const float* v) {
+    constexpr uint32_t kUnit = F <= 4 ? 4 / F : 1;  // entries per 16-byte unit
+    const uint32_t key = idx / kUnit;
+    uint32_t slot = (key * 2654435761u) >> 24;     // 8 bits: kDedupSlots == 256
+    while (true) {
+        const uint32_t prev = atomicCAS(keys + slot, kEmptyKey, key);
+        if (prev == kEmptyKey || prev == key) break;
+        slot = (slot + 1) & (kDedupSlots - 1);
+    }
+    const uint32_t off = (idx & (kUnit - 1)) * F;
+#pragma unroll
+    for (int f = 0; f < F; ++f) atomicAdd(vals + slot * 4 + off + f, v[f]);
+}
+
+template <int F, int BP, bool kDedup>
 __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const float* __restrict__ x,
                                                        const float* __restrict__ dout, int64_t N,
                                                        float* __restrict__ dtable) {
+    static_assert(!kDedup || F <= 4, "dedup units are 16 bytes");
     extern __shared__ __align__(16) float smem[];
     const int L = lp.L;
     const int W = L * F;
@@ -315,31 +459,67 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
     float* gs = smem + BP * 3;
     const int64_t p0 = (int64_t)blockIdx.x * BP;
     const int nvalid = (int)min((int64_t)BP, N - p0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+
+    uint32_t* keys = nullptr;
+    float* vals = nullptr;
+    if constexpr (kDedup) {
+        char* base = reinterpret_cast<char*>(smem + BP * 3 + BP * S);
+        keys = reinterpret_cast<uint32_t*>(base) + warp * kDedupSlots;
+        vals = reinterpret_cast<float*>(base + (size_t)nwarps * kDedupSlots * sizeof(uint32_t)) +
+               warp * kDedupSlots * 4;
+        for (int s = lane; s < kDedupSlots; s += 32) {
+            keys[s] = kEmptyKey;
+            *reinterpret_cast<float4*>(vals + s * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
 
     for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = __ldcs(x + p0 * 3 + i);
     stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
     __syncthreads();
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarps = blockDim.x >> 5;
     const int items = (BP / 32) * L;
     for (int it = warp; it < items; it += nwarps) {
         const int q = it / L;
         const int l = it - q * L;
         const int pl = q * 32 + lane;
+        float* dl = dtable + (uint64_t)l * lp.T * F;
         if (pl < nvalid) {
             Corners cr;
             locate_corners(xs[pl * 3 + 0], xs[pl * 3 + 1], xs[pl * 3 + 2], lp.scale[l], lp.mask, cr);
             float g[F];
             load_smem_entry<F>(gs + pl * S + l * F, g);
-            float* dl = dtable + (uint64_t)l * lp.T * F;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float v[F];
+            for (int qq = 0; qq < 4; ++qq) {
+                float va[F], vb[F];
 #pragma unroll
-                for (int f = 0; f < F; ++f) v[f] = cr.w[c] * g[f];
-                RedAdd<F>::add(dl + (uint64_t)cr.idx[c] * F, v);
+                for (int f = 0; f < F; ++f) {
+                    va[f] = cr.w[2 * qq] * g[f];
+                    vb[f] = cr.w[2 * qq + 1] * g[f];
+                }
+                if constexpr (kDedup) {
+                    dedup_add<F>(keys, vals, cr.idx[2 * qq], va);
+                    dedup_add<F>(keys, vals, cr.idx[2 * qq + 1], vb);
+                } else {
+                    red_pair<F>(dl, cr.idx[2 * qq], cr.idx[2 * qq + 1], va, vb);
+                }
             }
+        }
+        if constexpr (kDedup) {
+            constexpr uint32_t kUnit = F <= 4 ? 4 / F : 1;
+            __syncwarp();
+            for (int s = lane; s < kDedupSlots; s += 32) {
+                const uint32_t key = keys[s];
+                if (key != kEmptyKey) {
+                    float4 v = *reinterpret_cast<float4*>(vals + s * 4);
+                    float u[4] = {v.x, v.y, v.z, v.w};
+                    RedAdd<4>::add(dl + (uint64_t)key * kUnit * F, u);
+                    keys[s] = kEmptyKey;
+                    *reinterpret_cast<float4*>(vals + s * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            __syncwarp();
         }
     }
 }

@@ -97,6 +97,27 @@ def test_create_rejects_invalid(args):
     assert e.value.code == hg.HASHGRID_ERR_ARG
 
 
+def test_options():
+    h = hg.hashgrid_create(16, 2, 19, 16, 512)
+    try:
+        assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_FORWARD_GATHER) == hg.HASHGRID_GATHER_AUTO
+        assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_BACKWARD_MODE) == hg.HASHGRID_BACKWARD_AUTO
+        hg.hashgrid_set_option(h, hg.HASHGRID_OPT_FORWARD_GATHER, hg.HASHGRID_GATHER_SECTOR)
+        hg.hashgrid_set_option(h, hg.HASHGRID_OPT_BACKWARD_MODE, hg.HASHGRID_BACKWARD_WARP_DEDUP)
+        assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_FORWARD_GATHER) == hg.HASHGRID_GATHER_SECTOR
+        assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_BACKWARD_MODE) == hg.HASHGRID_BACKWARD_WARP_DEDUP
+        for opt, val in [(hg.HASHGRID_OPT_FORWARD_GATHER, 3), (hg.HASHGRID_OPT_BACKWARD_MODE, -1), (7, 0)]:
+            assert hg.lib.hashgrid_set_option(h, opt, val) == hg.HASHGRID_ERR_ARG
+        assert hg.lib.hashgrid_set_option(None, 0, 0) == hg.HASHGRID_ERR_ARG
+    finally:
+        hg.hashgrid_destroy(h)
+    h8 = hg.hashgrid_create(4, 8, 10, 2, 16)
+    try:   # warp dedup works on 16-byte gradient units: F <= 4 only
+        assert hg.lib.hashgrid_set_option(h8, hg.HASHGRID_OPT_BACKWARD_MODE, hg.HASHGRID_BACKWARD_WARP_DEDUP) == hg.HASHGRID_ERR_ARG
+    finally:
+        hg.hashgrid_destroy(h8)
+
+
 def test_calls_validate_before_any_launch():
     h = hg.hashgrid_create(4, 2, 10, 2, 16)
     try:

@@ -39,11 +39,20 @@ def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def make_pair(L, F, log2T, N_min, N_max, dtype="f32"):
+# every kernel variant (forward gather mode, backward reduction mode) is held to the same bars
+GATHERS = ["corner", "sector"]
+BACKWARDS = ["atomic", "dedup"]
+
+
+def make_pair(L, F, log2T, N_min, N_max, dtype="f32", gather="auto", backward="auto"):
     hg = hgmod()
     dt = hg.HASHGRID_F16 if dtype == "f16" else hg.HASHGRID_F32
-    return hg.HashGrid(L, F, log2T, N_min, N_max, dt), oracle.Grid(L, F, log2T, N_min, N_max,
-                                                                    oracle.F16 if dtype == "f16" else oracle.F32)
+    gm = {"auto": hg.HASHGRID_GATHER_AUTO, "corner": hg.HASHGRID_GATHER_CORNER,
+          "sector": hg.HASHGRID_GATHER_SECTOR}[gather]
+    bm = {"auto": hg.HASHGRID_BACKWARD_AUTO, "atomic": hg.HASHGRID_BACKWARD_ATOMIC,
+          "dedup": hg.HASHGRID_BACKWARD_WARP_DEDUP if F <= 4 else hg.HASHGRID_BACKWARD_ATOMIC}[backward]
+    return (hg.HashGrid(L, F, log2T, N_min, N_max, dt, forward_gather=gm, backward_mode=bm),
+            oracle.Grid(L, F, log2T, N_min, N_max, oracle.F16 if dtype == "f16" else oracle.F32))
 
 
 def gpu_forward(grid, x, table):
@@ -109,18 +118,20 @@ def test_indices_bit_exact(name, reduced_inputs):
     np.testing.assert_array_equal(got, want)
 
 
+@pytest.mark.parametrize("gather", GATHERS)
 @pytest.mark.parametrize("name", list(workloads.WORKLOADS))
-def test_forward_parity(name, reduced_inputs):
+def test_forward_parity(name, gather, reduced_inputs):
     w, inp = reduced_inputs(name)
-    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, gather=gather)
     got = gpu_forward(grid, inp.x, inp.table)
     check_forward(og, inp.x, inp.table, got, w.dtype)
 
 
+@pytest.mark.parametrize("mode", BACKWARDS)
 @pytest.mark.parametrize("name", list(workloads.WORKLOADS))
-def test_backward_parity(name, reduced_inputs):
+def test_backward_parity(name, mode, reduced_inputs):
     w, inp = reduced_inputs(name)
-    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, backward=mode)
     got = gpu_backward(grid, inp.x, inp.g)
     ref = og.backward(inp.x, inp.g, nthreads=THREADS)
     assert rel_l2(got, ref) <= BWD_REL_L2
@@ -140,11 +151,12 @@ FULL_LEVELS = {   # gradient levels the oracle recomputes at full size (bounded 
 }
 
 
+@pytest.mark.parametrize("modes", [("auto", "auto"), ("corner", "dedup")])
 @pytest.mark.parametrize("name", list(workloads.WORKLOADS))
-def test_full_size(name):
+def test_full_size(name, modes):
     w = workloads.WORKLOADS[name]
     inp = workloads.make_inputs(w, seed=0, grads=True)
-    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, gather=modes[0], backward=modes[1])
     x_d, t_d, g_d = dev(inp.x), dev(inp.table), dev(inp.g)
     out_d = grid.forward(x_d, t_d)
     dt_d = grid.backward(x_d, g_d)
@@ -173,9 +185,10 @@ def test_full_size(name):
 # Edge cases
 # ---------------------------------------------------------------------------------------
 
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup")])
 @pytest.mark.parametrize("N", [1, 2, 31, 32, 33, 63, 64, 65, 127, 129, 1000])
-def test_ragged_batch_sizes(N):
-    grid, og = make_pair(16, 2, 19, 16, 512)
+def test_ragged_batch_sizes(N, modes):
+    grid, og = make_pair(16, 2, 19, 16, 512, gather=modes[0], backward=modes[1])
     rng = np.random.default_rng(N)
     table = workloads.table_values(rng, 16, 2**19, 2)
     x = workloads.uniform_points(rng, N)
@@ -184,10 +197,11 @@ def test_ragged_batch_sizes(N):
     assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g, nthreads=THREADS)) <= BWD_REL_L2
 
 
-def test_special_coordinates():
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup")])
+def test_special_coordinates(modes):
     """x = 0, the largest fp32 below 1, exactly 1 (voxel N_l, corner N_l + 1), points
     outside the cube (no clamping), and grid vertices (bit-exact table entries)."""
-    grid, og = make_pair(4, 2, 10, 2, 16)
+    grid, og = make_pair(4, 2, 10, 2, 16, gather=modes[0], backward=modes[1])
     rng = np.random.default_rng(5)
     table = rng.standard_normal((4, 1024, 2)).astype(np.float32)
     vals = np.array([0.0, 1.0 - 2**-24, 1.0, 0.5, 0.25, -0.3, 1.7, -2.0, 3.25], dtype=np.float32)
@@ -203,10 +217,11 @@ def test_special_coordinates():
     assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g)) <= BWD_REL_L2
 
 
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup")])
 @pytest.mark.parametrize("F", [1, 2, 4, 8])
 @pytest.mark.parametrize("dtype", ["f32", "f16"])
-def test_feature_widths_and_dtypes(F, dtype):
-    grid, og = make_pair(5, F, 12, 3, 200, dtype)
+def test_feature_widths_and_dtypes(F, dtype, modes):
+    grid, og = make_pair(5, F, 12, 3, 200, dtype, gather=modes[0], backward=modes[1])
     rng = np.random.default_rng(F)
     table = workloads.table_values(rng, 5, 2**12, F, dtype)
     x = workloads.uniform_points(rng, 3000)
@@ -222,9 +237,10 @@ def test_feature_widths_and_dtypes(F, dtype):
     (2, 1, 24, 512, 2**16),      # largest table
     (32, 8, 8, 2, 300),          # widest output row (256 floats, > 48 KB of shared memory)
 ])
-def test_extreme_shapes(shape):
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup")])
+def test_extreme_shapes(shape, modes):
     L, F, log2T, a, b = shape
-    grid, og = make_pair(L, F, log2T, a, b)
+    grid, og = make_pair(L, F, log2T, a, b, gather=modes[0], backward=modes[1])
     rng = np.random.default_rng(L * 100 + F)
     table = workloads.table_values(rng, L, 2**log2T, F)
     x = workloads.uniform_points(rng, 777)
@@ -250,6 +266,28 @@ def test_backward_accumulates_and_side_stream():
     ref = og.backward(inp.x, inp.g, nthreads=THREADS)
     assert rel_l2(d.cpu().numpy(), 2 * ref) <= BWD_REL_L2
     check_forward(og, inp.x, inp.table, out.cpu().numpy(), "f32")
+
+
+def test_sector_gather_alignment():
+    """AUTO falls back to per-corner gathers for a table that is only 16-byte aligned;
+    forcing sector gathers on it is an alignment error (no launch)."""
+    hg = hgmod()
+    grid, og = make_pair(4, 2, 10, 2, 16)
+    rng = np.random.default_rng(8)
+    table = rng.standard_normal((4, 1024, 2)).astype(np.float32)
+    x = rng.random((500, 3), dtype=np.float32)
+    buf = torch.zeros(4 * 1024 * 2 + 4, device="cuda")
+    t16 = buf[4:]                                     # 16 bytes past a 512-byte boundary
+    assert t16.data_ptr() % 32 == 16
+    t16.copy_(torch.from_numpy(table.ravel()).cuda())
+    out = grid.forward(dev(x), t16)
+    torch.cuda.synchronize()
+    check_forward(og, x, table, out.cpu().numpy(), "f32")
+    hg.hashgrid_set_option(grid.handle, hg.HASHGRID_OPT_FORWARD_GATHER, hg.HASHGRID_GATHER_SECTOR)
+    o2 = torch.full((500, 8), 3.0, device="cuda")
+    rc = hg.lib.hashgrid_forward(grid.handle, dev(x).data_ptr(), 500, t16.data_ptr(), o2.data_ptr(), None)
+    torch.cuda.synchronize()
+    assert rc == hg.HASHGRID_ERR_ALIGN and bool(torch.all(o2 == 3.0))
 
 
 def test_errors_on_device():
