@@ -163,7 +163,9 @@ const char *hashgrid_last_error(void);
  *     ([NeRFace-HG] section 2: primes (1, 2654435761, 805459861)); the second corner is
  *     loaded separately only when it is not in that sector. Needs a 32-byte-aligned table
  *     (HASHGRID_ERR_ALIGN otherwise);
- *   HASHGRID_GATHER_AUTO: SECTOR when the table is 32-byte aligned, else CORNER.
+ *   HASHGRID_GATHER_AUTO: CORNER (on B200 the L1 already merges the second corner's
+ *     request when it falls in the sector just requested, and per-corner loads leave room
+ *     for more warps; CORNER measured as fast or faster on every workload tested).
  * HASHGRID_OPT_BACKWARD_MODE -- how the backward pass reduces into dL_dtable:
  *   HASHGRID_BACKWARD_ATOMIC: each (point, level) reduces its 8 corner contributions, the
  *     two x-corners merged into one 16-byte reduction when they share an aligned unit;
@@ -171,7 +173,9 @@ const char *hashgrid_last_error(void);
  *     its contributions per distinct 16-byte gradient unit in shared memory, then issues one
  *     reduction per unit. Pays off for coherent batches (consecutive samples along rays)
  *     where neighbouring points share corners. Needs F <= 4;
- *   HASHGRID_BACKWARD_AUTO: ATOMIC.
+ *   HASHGRID_BACKWARD_AUTO: per warp and level, WARP_DEDUP when at least half of the
+ *     warp's points lie in a voxel adjacent to the previous point's voxel (they can share
+ *     corners), else ATOMIC. F = 8 always uses ATOMIC.
  * Returns HASHGRID_ERR_ARG for an unknown option or value.
  */
 enum hashgrid_option { HASHGRID_OPT_FORWARD_GATHER = 0, HASHGRID_OPT_BACKWARD_MODE = 1 };

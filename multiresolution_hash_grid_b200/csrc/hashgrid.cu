@@ -174,12 +174,15 @@ int launch_forward(const hashgrid_s* h, const float* x, int64_t N, const void* t
     return launch_status("forward");
 }
 
-template <int F, bool kDedup>
+template <int F, int kMode>
 int launch_backward_mode(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
                          float* dtable, cudaStream_t s) {
-    auto k = hg::backward_kernel<F, kTile, kDedup>;
-    const int threads = tile_threads(h->L);
-    const size_t smem = hg::tile_smem_bytes(kTile, h->L, F) + (kDedup ? hg::dedup_smem_bytes(threads / 32) : 0);
+    auto k = hg::backward_kernel<F, kTile, kMode>;
+    // Grouping modes keep 7-13 KB of shared memory per warp: 8 warps per block.
+    const int threads = kMode == hg::kAtomicOnly ? tile_threads(h->L)
+                                                  : (tile_threads(h->L) < 256 ? tile_threads(h->L) : 256);
+    const size_t smem = hg::tile_smem_bytes(kTile, h->L, F) +
+                        (kMode == hg::kAtomicOnly ? 0 : hg::group_smem_bytes(threads / 32, F));
     if (int rc = prepare_smem(k, smem)) return rc;
     const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
     k<<<blocks, threads, smem, s>>>(h->lp, x, dout, N, dtable);
@@ -191,9 +194,11 @@ int launch_backward(const hashgrid_s* h, const float* x, const float* dout, int6
                     float* dtable, cudaStream_t s) {
     if constexpr (F <= 4) {
         if (h->backward_mode == HASHGRID_BACKWARD_WARP_DEDUP)
-            return launch_backward_mode<F, true>(h, x, dout, N, dtable, s);
+            return launch_backward_mode<F, hg::kGroupAlways>(h, x, dout, N, dtable, s);
+        if (h->backward_mode == HASHGRID_BACKWARD_AUTO)
+            return launch_backward_mode<F, hg::kAdaptive>(h, x, dout, N, dtable, s);
     }
-    return launch_backward_mode<F, false>(h, x, dout, N, dtable, s);
+    return launch_backward_mode<F, hg::kAtomicOnly>(h, x, dout, N, dtable, s);
 }
 
 size_t table_bytes(const hashgrid_s* h) {
@@ -306,7 +311,7 @@ int hashgrid_forward(hashgrid_t h, const float* x, int64_t N, const void* table,
     const bool half = h->dtype == HASHGRID_F16;
     // Sector gathers issue 256-bit loads, which need a 32-byte-aligned table.
     const bool aligned32 = reinterpret_cast<uintptr_t>(table) % 32 == 0;
-    bool sector = h->forward_gather != HASHGRID_GATHER_CORNER && aligned32;
+    const bool sector = h->forward_gather == HASHGRID_GATHER_SECTOR;
     if (h->forward_gather == HASHGRID_GATHER_SECTOR && !aligned32)
         return fail(HASHGRID_ERR_ALIGN, "sector gathers need a 32-byte-aligned table (%p)", table);
     switch (h->F) {

@@ -225,6 +225,7 @@ __device__ __forceinline__ void red_pair(float* dl, uint32_t a, uint32_t b, cons
 struct Corners {
     uint32_t idx[8];
     float w[8];
+    int v[3];  // the voxel (lower corner)
 };
 
 __device__ __forceinline__ void locate_corners(float x0, float x1, float x2, float scale,
@@ -235,6 +236,9 @@ __device__ __forceinline__ void locate_corners(float x0, float x1, float x2, flo
     const int v0 = __float2int_rd(xs0);
     const int v1 = __float2int_rd(xs1);
     const int v2 = __float2int_rd(xs2);
+    cr.v[0] = v0;
+    cr.v[1] = v1;
+    cr.v[2] = v2;
     const float f0 = __fsub_rn(xs0, __int2float_rn(v0));
     const float f1 = __fsub_rn(xs1, __int2float_rn(v1));
     const float f2 = __fsub_rn(xs2, __int2float_rn(v2));
@@ -367,8 +371,16 @@ __device__ __forceinline__ void gather_corners(const TT* __restrict__ tl, const 
     }
 }
 
+// Per-corner gathers run 3 blocks of 512 threads per SM (<= 42 registers: more warps keep
+// more gathers in flight, measured 10-15% faster than the compiler's own choice); sector
+// gathers and F = 8 need more registers: 2 blocks per SM (<= 64 registers), and one
+// block for sector gathers of F = 8.
+__host__ __device__ constexpr int forward_min_blocks(int F, bool sector) {
+    return sector ? (F == 8 ? 1 : 2) : (F == 8 ? 2 : 3);
+}
+
 template <int F, typename TT, int BP, bool kSector>
-__global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const float* __restrict__ x,
+__global__ void __launch_bounds__(512, forward_min_blocks(F, kSector)) forward_kernel(LevelParams lp, const float* __restrict__ x,
                                                       int64_t N, const TT* __restrict__ table,
                                                       float* __restrict__ out) {
     extern __shared__ __align__(16) float smem[];
@@ -412,45 +424,108 @@ __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const floa
 }
 
 // ---------------------------------------------------------------------------------------
-// Backward kernel (table gradient). Grid: one block per BP-point tile.
+// Backward kernel (table gradient). Grid: one block per BP-point tile. Each (point, level,
+// corner) contributes w_c * dL_dout[p][l*F..] to the level's gradient table.
 //
-// kDedup = false: each lane reduces its own 8 contributions w_c * g into the level's
-// gradient table, the two x-corners of an edge merged into one 16-byte red when they share
-// an aligned unit (red_pair).
+// Grouped reductions (coherent batches, e.g. consecutive samples along rays): a warp first
+// groups its 32 x 8 contributions by 16-byte gradient unit, then issues one red.v4 per
+// distinct unit. Consecutive samples of a ray share voxels at coarse levels and voxel faces
+// at finer ones, so far fewer reductions reach L2, whose reduction rate bounds this pass.
+// Grouping uses only integer shared-memory atomics (native; fp32 shared-memory atomics are
+// compare-and-swap loops that serialise when lanes collide): a direct-mapped table of 512
+// slots maps unit keys to slots (atomicCAS; a contribution whose slot already holds another
+// key is reduced on its own right away, so there is no probing), each grouped contribution
+// is pushed onto its slot's list (atomicExch), and after a warp barrier each lane walks the
+// lists of its slots, summing in registers.
 //
-// kDedup = true (coherent batches, e.g. consecutive samples along rays): a warp first sums
-// its 32 x 8 contributions per 16-byte gradient unit in a shared-memory open-addressing
-// table (keys = unit index within the level, 256 slots, values = 4 fp32), then issues one
-// red.v4 per distinct unit. Consecutive samples of a ray share voxels at coarse levels and
-// voxel faces at finer ones, so far fewer reductions reach L2.
+// Backward modes: kAtomicOnly -- every (point, level) reduces its own 8 contributions, the
+// two x-corners of an edge merged into one 16-byte red when they share an aligned unit
+// (red_pair). kGroupAlways -- every warp item is grouped. kAdaptive -- a warp item is
+// grouped when at least half of its lanes sit in a voxel adjacent to (or equal to) the
+// previous lane's voxel, i.e. when neighbouring points can share corners; otherwise it
+// takes the kAtomicOnly path (uniformly scattered points never share corners in a warp).
 // ---------------------------------------------------------------------------------------
-constexpr int kDedupSlots = 256;
-constexpr uint32_t kEmptyKey = 0xffffffffu;
+enum BackwardMode { kAtomicOnly = 0, kAdaptive = 1, kGroupAlways = 2 };
 
-__host__ __device__ constexpr size_t dedup_smem_bytes(int warps) {
-    return (size_t)warps * kDedupSlots * (sizeof(uint32_t) + 4 * sizeof(float));
+constexpr int kGroupSlots = 512;
+constexpr int kGroupItems = 256;           // 32 lanes x 8 corners
+constexpr uint32_t kEmpty = 0xffffffffu;
+constexpr uint32_t kEnd = 0xffffu;
+
+// Shared memory of one warp: keys[512], head[512], next[256] (u32), values[256 * F] (f32).
+__host__ __device__ constexpr size_t group_smem_bytes(int warps, int F) {
+    return (size_t)warps * (2 * kGroupSlots * sizeof(uint32_t) +
+                            (size_t)kGroupItems * (sizeof(uint32_t) + (size_t)F * sizeof(float)));
 }
 
 template <int F>
-__device__ __forceinline__ void dedup_add(uint32_t* keys, float* vals, uint32_t idx, const float* v) {
-    constexpr uint32_t kUnit = F <= 4 ? 4 / F : 1;  // entries per 16-byte unit
-    const uint32_t key = idx / kUnit;
-    uint32_t slot = (key * 2654435761u) >> 24;     // 8 bits: kDedupSlots == 256
-    while (true) {
-        const uint32_t prev = atomicCAS(keys + slot, kEmptyKey, key);
-        if (prev == kEmptyKey || prev == key) break;
-        slot = (slot + 1) & (kDedupSlots - 1);
-    }
-    const uint32_t off = (idx & (kUnit - 1)) * F;
-#pragma unroll
-    for (int f = 0; f < F; ++f) atomicAdd(vals + slot * 4 + off + f, v[f]);
-}
+struct GroupWarp {
+    static constexpr uint32_t kUnit = 4 / F;  // table entries per 16-byte unit
+    uint32_t* keys;
+    uint32_t* head;
+    uint32_t* next;
+    float* vals;
 
-template <int F, int BP, bool kDedup>
+    __device__ __forceinline__ GroupWarp(char* base, int warp) {
+        char* w = base + (size_t)warp * group_smem_bytes(1, F);
+        keys = reinterpret_cast<uint32_t*>(w);
+        head = keys + kGroupSlots;
+        next = head + kGroupSlots;
+        vals = reinterpret_cast<float*>(next + kGroupItems);
+    }
+
+    __device__ __forceinline__ void clear(int lane) {
+        for (int s = lane; s < kGroupSlots; s += 32) {
+            keys[s] = kEmpty;
+            head[s] = kEmpty;
+        }
+    }
+
+    // Contribution `id` (lane * 8 + corner) of value v to table entry idx of level table dl.
+    __device__ __forceinline__ void push(float* dl, uint32_t idx, uint32_t id, const float* v) {
+        const uint32_t key = idx / kUnit;
+        const uint32_t slot = (key * 2654435761u) >> 23;  // 9 bits: kGroupSlots == 512
+        const uint32_t prev = atomicCAS(keys + slot, kEmpty, key);
+        if (prev != kEmpty && prev != key) {  // slot taken by another unit: reduce directly
+            RedAdd<F>::add(dl + (uint64_t)idx * F, v);
+            return;
+        }
+#pragma unroll
+        for (int f = 0; f < F; ++f) vals[id * F + f] = v[f];
+        const uint32_t old = atomicExch(head + slot, id);
+        next[id] = (old & kEnd) | ((idx & (kUnit - 1)) << 16);
+    }
+
+    // After __syncwarp(): one red.v4 per occupied slot, then the slots are emptied.
+    __device__ __forceinline__ void flush(float* dl, int lane) {
+        for (int s = lane; s < kGroupSlots; s += 32) {
+            const uint32_t key = keys[s];
+            if (key == kEmpty) continue;
+            float u[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t id = head[s] & kEnd;
+            while (id != kEnd) {
+                const uint32_t n = next[id];
+                const uint32_t off = (n >> 16) * F;
+#pragma unroll
+                for (int f = 0; f < F; ++f) {
+                    const float v = vals[id * F + f];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) u[k] += (off + f == (uint32_t)k) ? v : 0.f;
+                }
+                id = n & kEnd;
+            }
+            RedAdd<4>::add(dl + (uint64_t)key * 4, u);
+            keys[s] = kEmpty;
+            head[s] = kEmpty;
+        }
+    }
+};
+
+template <int F, int BP, int kMode>
 __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const float* __restrict__ x,
                                                        const float* __restrict__ dout, int64_t N,
                                                        float* __restrict__ dtable) {
-    static_assert(!kDedup || F <= 4, "dedup units are 16 bytes");
+    static_assert(kMode == kAtomicOnly || F <= 4, "grouped units are 16 bytes");
     extern __shared__ __align__(16) float smem[];
     const int L = lp.L;
     const int W = L * F;
@@ -462,18 +537,9 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nwarps = blockDim.x >> 5;
 
-    uint32_t* keys = nullptr;
-    float* vals = nullptr;
-    if constexpr (kDedup) {
-        char* base = reinterpret_cast<char*>(smem + BP * 3 + BP * S);
-        keys = reinterpret_cast<uint32_t*>(base) + warp * kDedupSlots;
-        vals = reinterpret_cast<float*>(base + (size_t)nwarps * kDedupSlots * sizeof(uint32_t)) +
-               warp * kDedupSlots * 4;
-        for (int s = lane; s < kDedupSlots; s += 32) {
-            keys[s] = kEmptyKey;
-            *reinterpret_cast<float4*>(vals + s * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    }
+    constexpr int FG = F <= 4 ? F : 4;  // keeps GroupWarp instantiable for kAtomicOnly
+    GroupWarp<FG> grp(reinterpret_cast<char*>(smem + BP * 3 + BP * S), warp);
+    if constexpr (kMode != kAtomicOnly) grp.clear(lane);
 
     for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = __ldcs(x + p0 * 3 + i);
     stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
@@ -484,12 +550,37 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
         const int q = it / L;
         const int l = it - q * L;
         const int pl = q * 32 + lane;
+        const bool valid = pl < nvalid;
+        const int pc = valid ? pl : 0;  // rows past the tail read row 0 and contribute nothing
         float* dl = dtable + (uint64_t)l * lp.T * F;
-        if (pl < nvalid) {
-            Corners cr;
-            locate_corners(xs[pl * 3 + 0], xs[pl * 3 + 1], xs[pl * 3 + 2], lp.scale[l], lp.mask, cr);
-            float g[F];
-            load_smem_entry<F>(gs + pl * S + l * F, g);
+        Corners cr;
+        locate_corners(xs[pc * 3 + 0], xs[pc * 3 + 1], xs[pc * 3 + 2], lp.scale[l], lp.mask, cr);
+        float g[F];
+        load_smem_entry<F>(gs + pc * S + l * F, g);
+
+        bool group = (kMode == kGroupAlways);
+        if constexpr (kMode == kAdaptive) {
+            const int u0 = __shfl_up_sync(0xffffffffu, cr.v[0], 1);
+            const int u1 = __shfl_up_sync(0xffffffffu, cr.v[1], 1);
+            const int u2 = __shfl_up_sync(0xffffffffu, cr.v[2], 1);
+            const bool near = valid && lane > 0 && abs(cr.v[0] - u0) <= 1 && abs(cr.v[1] - u1) <= 1 &&
+                              abs(cr.v[2] - u2) <= 1;
+            group = __popc(__ballot_sync(0xffffffffu, near)) >= 16;
+        }
+        if (group) {
+            if (valid) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float v[F];
+#pragma unroll
+                    for (int f = 0; f < F; ++f) v[f] = cr.w[c] * g[f];
+                    grp.push(dl, cr.idx[c], lane * 8 + c, v);
+                }
+            }
+            __syncwarp();
+            grp.flush(dl, lane);
+            __syncwarp();
+        } else if (valid) {
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
                 float va[F], vb[F];
@@ -498,28 +589,8 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
                     va[f] = cr.w[2 * qq] * g[f];
                     vb[f] = cr.w[2 * qq + 1] * g[f];
                 }
-                if constexpr (kDedup) {
-                    dedup_add<F>(keys, vals, cr.idx[2 * qq], va);
-                    dedup_add<F>(keys, vals, cr.idx[2 * qq + 1], vb);
-                } else {
-                    red_pair<F>(dl, cr.idx[2 * qq], cr.idx[2 * qq + 1], va, vb);
-                }
+                red_pair<F>(dl, cr.idx[2 * qq], cr.idx[2 * qq + 1], va, vb);
             }
-        }
-        if constexpr (kDedup) {
-            constexpr uint32_t kUnit = F <= 4 ? 4 / F : 1;
-            __syncwarp();
-            for (int s = lane; s < kDedupSlots; s += 32) {
-                const uint32_t key = keys[s];
-                if (key != kEmptyKey) {
-                    float4 v = *reinterpret_cast<float4*>(vals + s * 4);
-                    float u[4] = {v.x, v.y, v.z, v.w};
-                    RedAdd<4>::add(dl + (uint64_t)key * kUnit * F, u);
-                    keys[s] = kEmptyKey;
-                    *reinterpret_cast<float4*>(vals + s * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
-            __syncwarp();
         }
     }
 }

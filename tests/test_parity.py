@@ -41,7 +41,7 @@ def dev(a):
 
 # every kernel variant (forward gather mode, backward reduction mode) is held to the same bars
 GATHERS = ["corner", "sector"]
-BACKWARDS = ["atomic", "dedup"]
+BACKWARDS = ["atomic", "auto", "dedup"]
 
 
 def make_pair(L, F, log2T, N_min, N_max, dtype="f32", gather="auto", backward="auto"):
@@ -185,7 +185,7 @@ def test_full_size(name, modes):
 # Edge cases
 # ---------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup")])
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto")])
 @pytest.mark.parametrize("N", [1, 2, 31, 32, 33, 63, 64, 65, 127, 129, 1000])
 def test_ragged_batch_sizes(N, modes):
     grid, og = make_pair(16, 2, 19, 16, 512, gather=modes[0], backward=modes[1])
@@ -197,7 +197,7 @@ def test_ragged_batch_sizes(N, modes):
     assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g, nthreads=THREADS)) <= BWD_REL_L2
 
 
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup")])
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto")])
 def test_special_coordinates(modes):
     """x = 0, the largest fp32 below 1, exactly 1 (voxel N_l, corner N_l + 1), points
     outside the cube (no clamping), and grid vertices (bit-exact table entries)."""
@@ -217,7 +217,7 @@ def test_special_coordinates(modes):
     assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g)) <= BWD_REL_L2
 
 
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup")])
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto")])
 @pytest.mark.parametrize("F", [1, 2, 4, 8])
 @pytest.mark.parametrize("dtype", ["f32", "f16"])
 def test_feature_widths_and_dtypes(F, dtype, modes):
@@ -237,7 +237,7 @@ def test_feature_widths_and_dtypes(F, dtype, modes):
     (2, 1, 24, 512, 2**16),      # largest table
     (32, 8, 8, 2, 300),          # widest output row (256 floats, > 48 KB of shared memory)
 ])
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup")])
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto")])
 def test_extreme_shapes(shape, modes):
     L, F, log2T, a, b = shape
     grid, og = make_pair(L, F, log2T, a, b, gather=modes[0], backward=modes[1])
