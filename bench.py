@@ -49,8 +49,8 @@ FLUSH_BYTES = 256 << 20
 CPU_SAMPLE_POINTS = 1 << 18
 REFERENCE_SAMPLE_POINTS = 1 << 15
 FALLBACK_HBM_GBS = 6650.0
-GATHER_MODES = {"auto": 0, "corner": 1, "sector": 2}          # HASHGRID_GATHER_*
-BACKWARD_MODES = {"auto": 0, "atomic": 1, "dedup": 2}        # HASHGRID_BACKWARD_*
+GATHER_MODES = {"auto": 0, "corner": 1, "sector": 2, "pair": 3}  # HASHGRID_GATHER_*
+BACKWARD_MODES = {"auto": 0, "atomic": 1, "dedup": 2, "runs": 3, "dedup_adaptive": 4}  # HASHGRID_BACKWARD_*
 
 
 # ---------------------------------------------------------------------------------------

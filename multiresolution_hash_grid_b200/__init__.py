@@ -34,9 +34,12 @@ HASHGRID_OPT_BACKWARD_MODE = 1
 HASHGRID_GATHER_AUTO = 0
 HASHGRID_GATHER_CORNER = 1
 HASHGRID_GATHER_SECTOR = 2
+HASHGRID_GATHER_PAIR = 3
 HASHGRID_BACKWARD_AUTO = 0
 HASHGRID_BACKWARD_ATOMIC = 1
 HASHGRID_BACKWARD_WARP_DEDUP = 2
+HASHGRID_BACKWARD_RUN_MERGE = 3
+HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE = 4
 
 
 class HashGridError(RuntimeError):

@@ -165,8 +165,10 @@ int prepare_smem(K kernel, size_t smem) {
 
 template <int F, typename TT>
 int launch_forward(const hashgrid_s* h, const float* x, int64_t N, const void* table, float* out,
-                   bool sector, cudaStream_t s) {
-    auto k = sector ? hg::forward_kernel<F, TT, kTile, true> : hg::forward_kernel<F, TT, kTile, false>;
+                   int gather, cudaStream_t s) {
+    auto k = gather == hg::kGatherSector ? hg::forward_kernel<F, TT, kTile, hg::kGatherSector>
+           : gather == hg::kGatherPair   ? hg::forward_kernel<F, TT, kTile, hg::kGatherPair>
+                                         : hg::forward_kernel<F, TT, kTile, hg::kGatherCorner>;
     const size_t smem = hg::tile_smem_bytes(kTile, h->L, F);
     if (int rc = prepare_smem(k, smem)) return rc;
     const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
@@ -177,15 +179,31 @@ int launch_forward(const hashgrid_s* h, const float* x, int64_t N, const void* t
 template <int F, int kMode>
 int launch_backward_mode(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
                          float* dtable, cudaStream_t s) {
-    auto k = hg::backward_kernel<F, kTile, kMode>;
-    // Grouping modes keep 7-13 KB of shared memory per warp: 8 warps per block.
-    const int threads = kMode == hg::kAtomicOnly ? tile_threads(h->L)
-                                                  : (tile_threads(h->L) < 256 ? tile_threads(h->L) : 256);
+    const int cap = hg::backward_threads(kMode);
+    const int threads = tile_threads(h->L) < cap ? tile_threads(h->L) : cap;
     const size_t smem = hg::tile_smem_bytes(kTile, h->L, F) +
                         (kMode == hg::kAtomicOnly ? 0 : hg::group_smem_bytes(threads / 32, F));
-    if (int rc = prepare_smem(k, smem)) return rc;
     const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
-    k<<<blocks, threads, smem, s>>>(h->lp, x, dout, N, dtable);
+    if constexpr (kMode == hg::kAtomicOnly) {
+        auto k = hg::backward_kernel_atomic<F, kTile>;
+        if (int rc = prepare_smem(k, smem)) return rc;
+        k<<<blocks, threads, smem, s>>>(h->lp, x, dout, N, dtable);
+    } else {
+        auto k = hg::backward_kernel_grouped<F, kTile, kMode>;
+        if (int rc = prepare_smem(k, smem)) return rc;
+        k<<<blocks, threads, smem, s>>>(h->lp, x, dout, N, dtable);
+    }
+    return launch_status("backward");
+}
+
+template <int F>
+int launch_backward_runs(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
+                         float* dtable, cudaStream_t s) {
+    auto k = hg::backward_kernel_runs<F>;
+    const size_t smem = hg::run_smem_bytes(h->L, F);
+    if (int rc = prepare_smem(k, smem)) return rc;
+    const unsigned blocks = (unsigned)((N + hg::kRunTile - 1) / hg::kRunTile);
+    k<<<blocks, 256, smem, s>>>(h->lp, x, dout, N, dtable);
     return launch_status("backward");
 }
 
@@ -193,9 +211,11 @@ template <int F>
 int launch_backward(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
                     float* dtable, cudaStream_t s) {
     if constexpr (F <= 4) {
+        if (h->backward_mode == HASHGRID_BACKWARD_RUN_MERGE || h->backward_mode == HASHGRID_BACKWARD_AUTO)
+            return launch_backward_runs<F>(h, x, dout, N, dtable, s);
         if (h->backward_mode == HASHGRID_BACKWARD_WARP_DEDUP)
             return launch_backward_mode<F, hg::kGroupAlways>(h, x, dout, N, dtable, s);
-        if (h->backward_mode == HASHGRID_BACKWARD_AUTO)
+        if (h->backward_mode == HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE)
             return launch_backward_mode<F, hg::kAdaptive>(h, x, dout, N, dtable, s);
     }
     return launch_backward_mode<F, hg::kAtomicOnly>(h, x, dout, N, dtable, s);
@@ -262,15 +282,16 @@ int hashgrid_set_option(hashgrid_t h, int option, int value) {
     if (int rc = check_handle(h)) return rc;
     switch (option) {
         case HASHGRID_OPT_FORWARD_GATHER:
-            if (value < HASHGRID_GATHER_AUTO || value > HASHGRID_GATHER_SECTOR)
+            if (value < HASHGRID_GATHER_AUTO || value > HASHGRID_GATHER_PAIR)
                 return fail(HASHGRID_ERR_ARG, "forward gather mode %d is not a HASHGRID_GATHER_* value", value);
             h->forward_gather = value;
             return ok();
         case HASHGRID_OPT_BACKWARD_MODE:
-            if (value < HASHGRID_BACKWARD_AUTO || value > HASHGRID_BACKWARD_WARP_DEDUP)
+            if (value < HASHGRID_BACKWARD_AUTO || value > HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE)
                 return fail(HASHGRID_ERR_ARG, "backward mode %d is not a HASHGRID_BACKWARD_* value", value);
-            if (value == HASHGRID_BACKWARD_WARP_DEDUP && h->F > 4)
-                return fail(HASHGRID_ERR_ARG, "warp dedup needs F <= 4 (16-byte gradient units), F = %d", h->F);
+            if ((value == HASHGRID_BACKWARD_WARP_DEDUP || value == HASHGRID_BACKWARD_RUN_MERGE ||
+                 value == HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE) && h->F > 4)
+                return fail(HASHGRID_ERR_ARG, "backward mode %d needs F <= 4, F = %d", value, h->F);
             h->backward_mode = value;
             return ok();
     }
@@ -311,9 +332,11 @@ int hashgrid_forward(hashgrid_t h, const float* x, int64_t N, const void* table,
     const bool half = h->dtype == HASHGRID_F16;
     // Sector gathers issue 256-bit loads, which need a 32-byte-aligned table.
     const bool aligned32 = reinterpret_cast<uintptr_t>(table) % 32 == 0;
-    const bool sector = h->forward_gather == HASHGRID_GATHER_SECTOR;
     if (h->forward_gather == HASHGRID_GATHER_SECTOR && !aligned32)
         return fail(HASHGRID_ERR_ALIGN, "sector gathers need a 32-byte-aligned table (%p)", table);
+    const int sector = h->forward_gather == HASHGRID_GATHER_SECTOR ? hg::kGatherSector
+                     : h->forward_gather == HASHGRID_GATHER_PAIR   ? hg::kGatherPair
+                                                                   : hg::kGatherCorner;
     switch (h->F) {
         case 1: return half ? launch_forward<1, __half>(h, x, N, table, out, sector, s) : launch_forward<1, float>(h, x, N, table, out, sector, s);
         case 2: return half ? launch_forward<2, __half>(h, x, N, table, out, sector, s) : launch_forward<2, float>(h, x, N, table, out, sector, s);

@@ -186,32 +186,46 @@ template <> struct RedAdd<8> {
     }
 };
 
-// Reduction of the x-corner pair (a, b) of one (y, z) edge: when both entries fall in the
-// same aligned 16-byte unit of the gradient table (F <= 2), one red.v4 carries both (the
-// unit's other elements receive +0.0, which leaves them unchanged); otherwise two F-wide
-// reductions are issued.
+// Reductions of the x-corner pair (a, b) of one (y, z) edge into level table dl, always
+// as 16-byte red.v4 instructions (L2 reduction throughput is per request, not per byte,
+// and uniform widths keep the warp's red instructions converged). For F <= 2 a 16-byte
+// unit holds 4 / F entries: when a and b share a unit (for F = 2: v0 even), one red.v4
+// carries both; otherwise each goes in its own unit, the unit's other elements receiving
+// +0.0, which leaves them unchanged. ra / rb say which of the two is reduced.
+template <int F>
+__device__ __forceinline__ void unit_vals(uint32_t i, const float* v, float (&u)[4]) {
+    constexpr uint32_t kUnit = 4 / F;
+    const uint32_t o = (i & (kUnit - 1)) * F;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        float t = 0.f;
+#pragma unroll
+        for (int f = 0; f < F; ++f) t = (o + f == (uint32_t)k) ? v[f] : t;
+        u[k] = t;
+    }
+}
+
 template <int F>
 __device__ __forceinline__ void red_pair(float* dl, uint32_t a, uint32_t b, const float* va,
-                                         const float* vb) {
+                                         const float* vb, bool ra = true, bool rb = true) {
     if constexpr (F <= 2) {
-        constexpr uint32_t kUnit = 4 / F;  // entries per 16-byte unit
-        if ((a ^ b) < kUnit) {
-            float u[4] = {0.f, 0.f, 0.f, 0.f};
-            const uint32_t oa = (a & (kUnit - 1)) * F, ob = (b & (kUnit - 1)) * F;
+        constexpr uint32_t kUnit = 4 / F;
+        const bool shared = ra && rb && (a ^ b) < kUnit;
+        float ua[4], ub[4];
+        unit_vals<F>(a, va, ua);
+        unit_vals<F>(b, vb, ub);
+        // first instruction: the shared unit, or a's unit, or (only b) b's unit
+        float u1[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-#pragma unroll
-                for (int f = 0; f < F; ++f) {
-                    if (oa + f == (uint32_t)k) u[k] += va[f];
-                    if (ob + f == (uint32_t)k) u[k] += vb[f];
-                }
-            }
-            RedAdd<4>::add(dl + (uint64_t)(a & ~(kUnit - 1)) * F, u);
-            return;
-        }
+        for (int k = 0; k < 4; ++k) u1[k] = shared ? ua[k] + ub[k] : (ra ? ua[k] : ub[k]);
+        const uint32_t i1 = ra ? a : b;
+        if (ra || rb) RedAdd<4>::add(dl + (uint64_t)(i1 & ~(kUnit - 1)) * F, u1);
+        // second instruction: b's own unit when both are reduced but do not share one
+        if (ra && rb && !shared) RedAdd<4>::add(dl + (uint64_t)(b & ~(kUnit - 1)) * F, ub);
+    } else {
+        if (ra) RedAdd<F>::add(dl + (uint64_t)a * F, va);
+        if (rb) RedAdd<F>::add(dl + (uint64_t)b * F, vb);
     }
-    RedAdd<F>::add(dl + (uint64_t)a * F, va);
-    RedAdd<F>::add(dl + (uint64_t)b * F, vb);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -337,16 +351,56 @@ __host__ __device__ constexpr size_t tile_smem_bytes(int BP, int L, int F) {
 
 // ---------------------------------------------------------------------------------------
 // Forward kernel. Grid: one block per BP-point tile.
-// kSector = false: one F-wide load per corner. kSector = true: one 256-bit sector load per
-// x-corner pair plus a predicated load of the second corner when it lies in another
-// sector (needs a 32-byte-aligned table).
+// kGatherCorner: one F-wide load per corner. kGatherSector: one 256-bit sector load per
+// x-corner pair plus a predicated load of the second corner when it lies in another sector
+// (needs a 32-byte-aligned table). kGatherPair: the same with 16-byte units (entries of at
+// most 8 bytes; wider entries load per corner).
 // ---------------------------------------------------------------------------------------
-template <int F, typename TT, bool kSector>
+enum GatherMode { kGatherCorner = 0, kGatherSector = 1, kGatherPair = 2 };
+
+// 16-byte read-only load.
+__device__ __forceinline__ void ld_unit(const void* p, uint32_t (&w)[4]) {
+    uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+}
+
+// Entry j of a loaded 16-byte unit (entries of at most 8 bytes: 16 / E entries per unit).
+template <int F, typename TT>
+__device__ __forceinline__ void unit_entry(const uint32_t (&w)[4], uint32_t j, float* e) {
+    constexpr int E = F * (int)sizeof(TT);
+    static_assert(E <= 8, "a 16-byte unit holds at least two entries");
+    uint32_t padded[8] = {w[0], w[1], w[2], w[3], w[0], w[1], w[2], w[3]};
+    // reuse the sector decoder on the first half: entries beyond the unit never occur
+    sector_entry<F, TT>(padded, j, e);
+}
+
+template <int F, typename TT, int kGather>
 __device__ __forceinline__ void gather_corners(const TT* __restrict__ tl, const Corners& cr,
                                                float (&e)[8][F]) {
-    if constexpr (!kSector) {
+    constexpr int E = F * (int)sizeof(TT);
+    if constexpr (kGather == kGatherCorner || (kGather == kGatherPair && E > 8)) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) EntryLoad<F, TT>::load(tl + (uint64_t)cr.idx[c] * F, e[c]);
+    } else if constexpr (kGather == kGatherPair) {
+        constexpr uint32_t kPer = 16 / E;  // entries per 16-byte unit
+        uint32_t w[4][4];
+        float far[4][F];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t a = cr.idx[2 * q], b = cr.idx[2 * q + 1];
+            ld_unit(tl + (uint64_t)(a & ~(kPer - 1)) * F, w[q]);
+            if ((a ^ b) >= kPer) EntryLoad<F, TT>::load(tl + (uint64_t)b * F, far[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t a = cr.idx[2 * q], b = cr.idx[2 * q + 1];
+            unit_entry<F, TT>(w[q], a & (kPer - 1), e[2 * q]);
+            float near[F];
+            unit_entry<F, TT>(w[q], b & (kPer - 1), near);
+            const bool same = (a ^ b) < kPer;
+#pragma unroll
+            for (int f = 0; f < F; ++f) e[2 * q + 1][f] = same ? near[f] : far[q][f];
+        }
     } else {
         using S = Sector<F, TT>;
         constexpr uint32_t kPer = S::kPerSector;
@@ -375,12 +429,12 @@ __device__ __forceinline__ void gather_corners(const TT* __restrict__ tl, const 
 // more gathers in flight, measured 10-15% faster than the compiler's own choice); sector
 // gathers and F = 8 need more registers: 2 blocks per SM (<= 64 registers), and one
 // block for sector gathers of F = 8.
-__host__ __device__ constexpr int forward_min_blocks(int F, bool sector) {
-    return sector ? (F == 8 ? 1 : 2) : (F == 8 ? 2 : 3);
+__host__ __device__ constexpr int forward_min_blocks(int F, int gather) {
+    return gather == kGatherSector ? (F == 8 ? 1 : 2) : (gather == kGatherPair || F == 8) ? 2 : 3;
 }
 
-template <int F, typename TT, int BP, bool kSector>
-__global__ void __launch_bounds__(512, forward_min_blocks(F, kSector)) forward_kernel(LevelParams lp, const float* __restrict__ x,
+template <int F, typename TT, int BP, int kGather>
+__global__ void __launch_bounds__(512, forward_min_blocks(F, kGather)) forward_kernel(LevelParams lp, const float* __restrict__ x,
                                                       int64_t N, const TT* __restrict__ table,
                                                       float* __restrict__ out) {
     extern __shared__ __align__(16) float smem[];
@@ -407,7 +461,7 @@ __global__ void __launch_bounds__(512, forward_min_blocks(F, kSector)) forward_k
             locate_corners(xs[pl * 3 + 0], xs[pl * 3 + 1], xs[pl * 3 + 2], lp.scale[l], lp.mask, cr);
             const TT* tl = table + (uint64_t)l * lp.T * F;
             float e[8][F];
-            gather_corners<F, TT, kSector>(tl, cr, e);
+            gather_corners<F, TT, kGather>(tl, cr, e);
             float o[F];
 #pragma unroll
             for (int f = 0; f < F; ++f) {
@@ -445,33 +499,37 @@ __global__ void __launch_bounds__(512, forward_min_blocks(F, kSector)) forward_k
 // previous lane's voxel, i.e. when neighbouring points can share corners; otherwise it
 // takes the kAtomicOnly path (uniformly scattered points never share corners in a warp).
 // ---------------------------------------------------------------------------------------
-enum BackwardMode { kAtomicOnly = 0, kAdaptive = 1, kGroupAlways = 2 };
+enum BackwardMode { kAtomicOnly = 0, kAdaptive = 1, kGroupAlways = 2, kRunMerge = 3 };
 
 constexpr int kGroupSlots = 512;
 constexpr int kGroupItems = 256;           // 32 lanes x 8 corners
 constexpr uint32_t kEmpty = 0xffffffffu;
 constexpr uint32_t kEnd = 0xffffu;
 
-// Shared memory of one warp: keys[512], head[512], next[256] (u32), values[256 * F] (f32).
+// Shared memory of one warp: keys[512], head[512], next[256], occupied[256] (u32),
+// values[F][256] (f32).
 __host__ __device__ constexpr size_t group_smem_bytes(int warps, int F) {
     return (size_t)warps * (2 * kGroupSlots * sizeof(uint32_t) +
-                            (size_t)kGroupItems * (sizeof(uint32_t) + (size_t)F * sizeof(float)));
+                            (size_t)kGroupItems * (2 * sizeof(uint32_t) + (size_t)F * sizeof(float)));
 }
 
 template <int F>
 struct GroupWarp {
     static constexpr uint32_t kUnit = 4 / F;  // table entries per 16-byte unit
-    uint32_t* keys;
-    uint32_t* head;
-    uint32_t* next;
-    float* vals;
+    uint32_t* keys;  // [kGroupSlots]
+    uint32_t* head;  // [kGroupSlots]
+    uint32_t* next;  // [kGroupItems], contribution id = corner * 32 + lane (conflict-free)
+    uint32_t* occ;   // [kGroupItems], slots claimed in this warp item, in claim order
+    float* vals;     // [F][kGroupItems] (structure of arrays: conflict-free)
+    uint32_t nocc;   // number of claimed slots (warp-uniform)
 
-    __device__ __forceinline__ GroupWarp(char* base, int warp) {
+    __device__ __forceinline__ GroupWarp(char* base, int warp) : nocc(0) {
         char* w = base + (size_t)warp * group_smem_bytes(1, F);
         keys = reinterpret_cast<uint32_t*>(w);
         head = keys + kGroupSlots;
         next = head + kGroupSlots;
-        vals = reinterpret_cast<float*>(next + kGroupItems);
+        occ = next + kGroupItems;
+        vals = reinterpret_cast<float*>(occ + kGroupItems);
     }
 
     __device__ __forceinline__ void clear(int lane) {
@@ -481,26 +539,54 @@ struct GroupWarp {
         }
     }
 
-    // Contribution `id` (lane * 8 + corner) of value v to table entry idx of level table dl.
-    __device__ __forceinline__ void push(float* dl, uint32_t idx, uint32_t id, const float* v) {
-        const uint32_t key = idx / kUnit;
-        const uint32_t slot = (key * 2654435761u) >> 23;  // 9 bits: kGroupSlots == 512
-        const uint32_t prev = atomicCAS(keys + slot, kEmpty, key);
-        if (prev != kEmpty && prev != key) {  // slot taken by another unit: reduce directly
-            RedAdd<F>::add(dl + (uint64_t)idx * F, v);
-            return;
-        }
+    // The lane's 8 contributions v[c] (F values each) to entries idx[c] of level table dl.
+    // The 8 slot claims and the 8 list pushes are each issued back to back.
+    // `vmask` is the ballot of the lanes that push (a prefix of the warp).
+    __device__ __forceinline__ void push8(float* dl, const uint32_t* idx, const float (*v)[F], int lane,
+                                          uint32_t vmask) {
+        uint32_t slot[8], prev[8];
 #pragma unroll
-        for (int f = 0; f < F; ++f) vals[id * F + f] = v[f];
-        const uint32_t old = atomicExch(head + slot, id);
-        next[id] = (old & kEnd) | ((idx & (kUnit - 1)) << 16);
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t key = idx[c] / kUnit;
+            slot[c] = (key * 2654435761u) >> 23;  // 9 bits: kGroupSlots == 512
+            prev[c] = atomicCAS(keys + slot[c], kEmpty, key);
+        }
+        // Record newly claimed slots (at most one claim per slot, <= 256 per item).
+        const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const bool claimed = prev[c] == kEmpty;
+            const uint32_t b = __ballot_sync(vmask, claimed);
+            if (claimed) occ[nocc + __popc(b & lt)] = slot[c];
+            nocc += __popc(b);
+        }
+        bool mine[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t key = idx[c] / kUnit;
+            mine[c] = prev[c] == kEmpty || prev[c] == key;
+            if (!mine[c]) {  // slot taken by another unit: reduce this one directly
+                RedAdd<F>::add(dl + (uint64_t)idx[c] * F, v[c]);
+            } else {
+#pragma unroll
+                for (int f = 0; f < F; ++f) vals[f * kGroupItems + c * 32 + lane] = v[c][f];
+            }
+        }
+        uint32_t old[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            if (mine[c]) old[c] = atomicExch(head + slot[c], (uint32_t)(c * 32 + lane));
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            if (mine[c]) next[c * 32 + lane] = (old[c] & kEnd) | ((idx[c] & (kUnit - 1)) << 16);
     }
 
-    // After __syncwarp(): one red.v4 per occupied slot, then the slots are emptied.
+    // After __syncwarp(): one red.v4 per claimed slot, then the slots are emptied.
     __device__ __forceinline__ void flush(float* dl, int lane) {
-        for (int s = lane; s < kGroupSlots; s += 32) {
+        nocc = __shfl_sync(0xffffffffu, nocc, 0);  // lanes past the tail did not push
+        for (uint32_t j = lane; j < nocc; j += 32) {
+            const uint32_t s = occ[j];
             const uint32_t key = keys[s];
-            if (key == kEmpty) continue;
             float u[4] = {0.f, 0.f, 0.f, 0.f};
             uint32_t id = head[s] & kEnd;
             while (id != kEnd) {
@@ -508,7 +594,7 @@ struct GroupWarp {
                 const uint32_t off = (n >> 16) * F;
 #pragma unroll
                 for (int f = 0; f < F; ++f) {
-                    const float v = vals[id * F + f];
+                    const float v = vals[f * kGroupItems + id];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) u[k] += (off + f == (uint32_t)k) ? v : 0.f;
                 }
@@ -518,13 +604,18 @@ struct GroupWarp {
             keys[s] = kEmpty;
             head[s] = kEmpty;
         }
+        nocc = 0;
     }
 };
 
+// Grouping modes run 8 warps per block (their tables take 8-10 KB of shared memory per
+// warp): 3 blocks per SM, 2 for F = 4. The plain mode runs 16 warps per block.
+__host__ __device__ constexpr int backward_threads(int mode) { return mode == kAtomicOnly ? 512 : 256; }
+
 template <int F, int BP, int kMode>
-__global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const float* __restrict__ x,
-                                                       const float* __restrict__ dout, int64_t N,
-                                                       float* __restrict__ dtable) {
+__device__ __forceinline__ void backward_body(const LevelParams& lp, const float* __restrict__ x,
+                                              const float* __restrict__ dout, int64_t N,
+                                              float* __restrict__ dtable) {
     static_assert(kMode == kAtomicOnly || F <= 4, "grouped units are 16 bytes");
     extern __shared__ __align__(16) float smem[];
     const int L = lp.L;
@@ -568,14 +659,14 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
             group = __popc(__ballot_sync(0xffffffffu, near)) >= 16;
         }
         if (group) {
+            const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
             if (valid) {
+                float v[8][FG];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float v[F];
+                for (int c = 0; c < 8; ++c)
 #pragma unroll
-                    for (int f = 0; f < F; ++f) v[f] = cr.w[c] * g[f];
-                    grp.push(dl, cr.idx[c], lane * 8 + c, v);
-                }
+                    for (int f = 0; f < FG; ++f) v[c][f] = cr.w[c] * g[f < F ? f : 0];
+                grp.push8(dl, cr.idx, v, lane, vmask);
             }
             __syncwarp();
             grp.flush(dl, lane);
@@ -592,6 +683,150 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
                 red_pair<F>(dl, cr.idx[2 * qq], cr.idx[2 * qq + 1], va, vb);
             }
         }
+    }
+}
+
+template <int F, int BP>
+__global__ void __launch_bounds__(512) backward_kernel_atomic(LevelParams lp, const float* __restrict__ x,
+                                                              const float* __restrict__ dout, int64_t N,
+                                                              float* __restrict__ dtable) {
+    backward_body<F, BP, kAtomicOnly>(lp, x, dout, N, dtable);
+}
+
+template <int F, int BP, int kMode>
+__global__ void __launch_bounds__(256, F == 4 ? 2 : 3) backward_kernel_grouped(LevelParams lp, const float* __restrict__ x,
+                                                                                const float* __restrict__ dout, int64_t N,
+                                                                                float* __restrict__ dtable) {
+    backward_body<F, BP, kMode>(lp, x, dout, N, dtable);
+}
+
+// ---------------------------------------------------------------------------------------
+// Run-merged backward (ordered batches, e.g. consecutive samples along rays). A lane walks a
+// run of kRun consecutive points at one level and keeps the current voxel's 8 corner sums
+// in registers. A point in the same voxel only adds to them. A step to a face-adjacent
+// voxel shares 4 corners: the 4 corners left behind are reduced into the table and the 4
+// shared ones carry their sums over. Any other step reduces all 8. Reductions of the two
+// x-corners of an edge are merged as in red_pair. Block: kRunTile points (32 runs) and 8
+// warps; a warp item is one level for the block's 32 runs.
+// Shared memory: x and the upstream-gradient rows, grouped by run with strides chosen so
+// that the lanes' row reads (lane = run) fall in distinct banks.
+// ---------------------------------------------------------------------------------------
+constexpr int kRun = 8;
+constexpr int kRunTile = 32 * kRun;
+
+__host__ __device__ constexpr int run_x_stride() { return kRun * 3 + 1; }
+__host__ __device__ constexpr int run_row_stride(int L, int F) { return L * F + row_pad(F); }
+__host__ __device__ constexpr int run_g_stride(int L, int F) { return kRun * run_row_stride(L, F) + F; }
+__host__ __device__ constexpr size_t run_smem_bytes(int L, int F) {
+    return sizeof(float) * ((size_t)32 * run_x_stride() + (size_t)32 * run_g_stride(L, F));
+}
+
+template <int F>
+__device__ __forceinline__ void run_flush(float* dl, const float (&acc)[8][F], const uint32_t (&cidx)[8],
+                                          int ax, uint32_t leave_bit) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int a = 2 * q, b = 2 * q + 1;
+        const bool fa = ax < 0 || (((uint32_t)a >> ax) & 1u) == leave_bit;
+        const bool fb = ax < 0 || (((uint32_t)b >> ax) & 1u) == leave_bit;
+        red_pair<F>(dl, cidx[a], cidx[b], acc[a], acc[b], fa, fb);
+    }
+}
+
+template <int F>
+__global__ void __launch_bounds__(256) backward_kernel_runs(LevelParams lp, const float* __restrict__ x,
+                                                           const float* __restrict__ dout, int64_t N,
+                                                           float* __restrict__ dtable) {
+    static_assert(F <= 4, "run merging keeps 8 x F sums in registers");
+    extern __shared__ __align__(16) float smem[];
+    const int L = lp.L;
+    const int W = L * F;
+    const int S = run_row_stride(L, F);
+    const int G = run_g_stride(L, F);
+    constexpr int XS = run_x_stride();
+    float* xs = smem;
+    float* gs = smem + 32 * XS;
+    const int64_t p0 = (int64_t)blockIdx.x * kRunTile;
+    const int nvalid = (int)min((int64_t)kRunTile, N - p0);
+
+    for (int k = threadIdx.x; k < nvalid * 3; k += blockDim.x) {
+        const int p = k / 3, i = k - 3 * (k / 3);
+        xs[(p / kRun) * XS + (p % kRun) * 3 + i] = __ldcs(x + p0 * 3 + k);
+    }
+    {
+        constexpr int V = F < 4 ? F : 4;
+        const int per_row = W / V;
+        const float* base = dout + p0 * (int64_t)W;
+        for (int k = threadIdx.x; k < nvalid * per_row; k += blockDim.x) {
+            const int row = k / per_row;
+            const int col = (k - row * per_row) * V;
+            float* dst = gs + (row / kRun) * G + (row % kRun) * S + col;
+            const float* src = base + (int64_t)row * W + col;
+            if constexpr (V == 4) {
+                *reinterpret_cast<float4*>(dst) = __ldcs(reinterpret_cast<const float4*>(src));
+            } else if constexpr (V == 2) {
+                *reinterpret_cast<float2*>(dst) = __ldcs(reinterpret_cast<const float2*>(src));
+            } else {
+                *dst = __ldcs(src);
+            }
+        }
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const int jmax = min(kRun, nvalid - lane * kRun);  // points of this lane's run (may be <= 0)
+    for (int l = warp; l < L; l += nwarps) {
+        float* dl = dtable + (uint64_t)l * lp.T * F;
+        float acc[8][F];
+        uint32_t cidx[8];
+        int cv0 = 0, cv1 = 0, cv2 = 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
+            for (int f = 0; f < F; ++f) acc[c][f] = 0.f;
+        for (int j = 0; j < jmax; ++j) {
+            const float* xp = xs + lane * XS + j * 3;
+            Corners cr;
+            locate_corners(xp[0], xp[1], xp[2], lp.scale[l], lp.mask, cr);
+            float g[F];
+            load_smem_entry<F>(gs + lane * G + j * S + l * F, g);
+            if (j > 0) {
+                const int dx = cr.v[0] - cv0, dy = cr.v[1] - cv1, dz = cr.v[2] - cv2;
+                if ((dx | dy | dz) != 0) {
+                    const bool face = abs(dx) + abs(dy) + abs(dz) == 1;
+                    const int ax = face ? (dx != 0 ? 0 : (dy != 0 ? 1 : 2)) : -1;
+                    const uint32_t leave_bit = (dx + dy + dz) > 0 ? 0u : 1u;
+                    run_flush<F>(dl, acc, cidx, ax, leave_bit);
+                    // carried corners: the new corner c with bit ax == leave_bit is the old
+                    // corner c ^ (1 << ax); every other new corner starts from zero
+                    float old[8][F];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+#pragma unroll
+                        for (int f = 0; f < F; ++f) old[c][f] = acc[c][f];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const bool keep = face && (((uint32_t)c >> ax) & 1u) == leave_bit;
+#pragma unroll
+                        for (int f = 0; f < F; ++f) {
+                            const float from = ax == 0 ? old[c ^ 1][f] : (ax == 1 ? old[c ^ 2][f] : old[c ^ 4][f]);
+                            acc[c][f] = keep ? from : 0.f;
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                cidx[c] = cr.idx[c];
+#pragma unroll
+                for (int f = 0; f < F; ++f) acc[c][f] = fmaf(cr.w[c], g[f], acc[c][f]);
+            }
+            cv0 = cr.v[0];
+            cv1 = cr.v[1];
+            cv2 = cr.v[2];
+        }
+        if (jmax > 0) run_flush<F>(dl, acc, cidx, -1, 0u);
     }
 }
 

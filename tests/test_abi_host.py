@@ -106,7 +106,7 @@ def test_options():
         hg.hashgrid_set_option(h, hg.HASHGRID_OPT_BACKWARD_MODE, hg.HASHGRID_BACKWARD_WARP_DEDUP)
         assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_FORWARD_GATHER) == hg.HASHGRID_GATHER_SECTOR
         assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_BACKWARD_MODE) == hg.HASHGRID_BACKWARD_WARP_DEDUP
-        for opt, val in [(hg.HASHGRID_OPT_FORWARD_GATHER, 3), (hg.HASHGRID_OPT_BACKWARD_MODE, -1), (7, 0)]:
+        for opt, val in [(hg.HASHGRID_OPT_FORWARD_GATHER, 4), (hg.HASHGRID_OPT_BACKWARD_MODE, -1), (hg.HASHGRID_OPT_BACKWARD_MODE, 5), (7, 0)]:
             assert hg.lib.hashgrid_set_option(h, opt, val) == hg.HASHGRID_ERR_ARG
         assert hg.lib.hashgrid_set_option(None, 0, 0) == hg.HASHGRID_ERR_ARG
     finally:
@@ -114,6 +114,7 @@ def test_options():
     h8 = hg.hashgrid_create(4, 8, 10, 2, 16)
     try:   # warp dedup works on 16-byte gradient units: F <= 4 only
         assert hg.lib.hashgrid_set_option(h8, hg.HASHGRID_OPT_BACKWARD_MODE, hg.HASHGRID_BACKWARD_WARP_DEDUP) == hg.HASHGRID_ERR_ARG
+        assert hg.lib.hashgrid_set_option(h8, hg.HASHGRID_OPT_BACKWARD_MODE, hg.HASHGRID_BACKWARD_RUN_MERGE) == hg.HASHGRID_ERR_ARG
     finally:
         hg.hashgrid_destroy(h8)
 

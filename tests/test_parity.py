@@ -40,17 +40,19 @@ def dev(a):
 
 
 # every kernel variant (forward gather mode, backward reduction mode) is held to the same bars
-GATHERS = ["corner", "sector"]
-BACKWARDS = ["atomic", "auto", "dedup"]
+GATHERS = ["corner", "sector", "pair"]
+BACKWARDS = ["atomic", "auto", "dedup", "runs", "dedup_adaptive"]
 
 
 def make_pair(L, F, log2T, N_min, N_max, dtype="f32", gather="auto", backward="auto"):
     hg = hgmod()
     dt = hg.HASHGRID_F16 if dtype == "f16" else hg.HASHGRID_F32
     gm = {"auto": hg.HASHGRID_GATHER_AUTO, "corner": hg.HASHGRID_GATHER_CORNER,
-          "sector": hg.HASHGRID_GATHER_SECTOR}[gather]
+          "sector": hg.HASHGRID_GATHER_SECTOR, "pair": hg.HASHGRID_GATHER_PAIR}[gather]
     bm = {"auto": hg.HASHGRID_BACKWARD_AUTO, "atomic": hg.HASHGRID_BACKWARD_ATOMIC,
-          "dedup": hg.HASHGRID_BACKWARD_WARP_DEDUP if F <= 4 else hg.HASHGRID_BACKWARD_ATOMIC}[backward]
+          "dedup": hg.HASHGRID_BACKWARD_WARP_DEDUP if F <= 4 else hg.HASHGRID_BACKWARD_ATOMIC,
+          "runs": hg.HASHGRID_BACKWARD_RUN_MERGE if F <= 4 else hg.HASHGRID_BACKWARD_ATOMIC,
+          "dedup_adaptive": hg.HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE if F <= 4 else hg.HASHGRID_BACKWARD_ATOMIC}[backward]
     return (hg.HashGrid(L, F, log2T, N_min, N_max, dt, forward_gather=gm, backward_mode=bm),
             oracle.Grid(L, F, log2T, N_min, N_max, oracle.F16 if dtype == "f16" else oracle.F32))
 
@@ -151,7 +153,7 @@ FULL_LEVELS = {   # gradient levels the oracle recomputes at full size (bounded 
 }
 
 
-@pytest.mark.parametrize("modes", [("auto", "auto"), ("corner", "dedup")])
+@pytest.mark.parametrize("modes", [("auto", "auto"), ("corner", "dedup"), ("sector", "runs")])
 @pytest.mark.parametrize("name", list(workloads.WORKLOADS))
 def test_full_size(name, modes):
     w = workloads.WORKLOADS[name]
@@ -185,7 +187,7 @@ def test_full_size(name, modes):
 # Edge cases
 # ---------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto")])
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto"), ("pair", "runs")])
 @pytest.mark.parametrize("N", [1, 2, 31, 32, 33, 63, 64, 65, 127, 129, 1000])
 def test_ragged_batch_sizes(N, modes):
     grid, og = make_pair(16, 2, 19, 16, 512, gather=modes[0], backward=modes[1])
@@ -197,7 +199,7 @@ def test_ragged_batch_sizes(N, modes):
     assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g, nthreads=THREADS)) <= BWD_REL_L2
 
 
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto")])
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto"), ("pair", "runs")])
 def test_special_coordinates(modes):
     """x = 0, the largest fp32 below 1, exactly 1 (voxel N_l, corner N_l + 1), points
     outside the cube (no clamping), and grid vertices (bit-exact table entries)."""
@@ -217,7 +219,7 @@ def test_special_coordinates(modes):
     assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g)) <= BWD_REL_L2
 
 
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto")])
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto"), ("pair", "runs")])
 @pytest.mark.parametrize("F", [1, 2, 4, 8])
 @pytest.mark.parametrize("dtype", ["f32", "f16"])
 def test_feature_widths_and_dtypes(F, dtype, modes):
@@ -237,7 +239,7 @@ def test_feature_widths_and_dtypes(F, dtype, modes):
     (2, 1, 24, 512, 2**16),      # largest table
     (32, 8, 8, 2, 300),          # widest output row (256 floats, > 48 KB of shared memory)
 ])
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto")])
+@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto"), ("pair", "runs")])
 def test_extreme_shapes(shape, modes):
     L, F, log2T, a, b = shape
     grid, og = make_pair(L, F, log2T, a, b, gather=modes[0], backward=modes[1])
