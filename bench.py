@@ -50,6 +50,7 @@ CPU_SAMPLE_POINTS = 1 << 18
 REFERENCE_SAMPLE_POINTS = 1 << 15
 FALLBACK_HBM_GBS = 6650.0
 GATHER_MODES = {"auto": 0, "corner": 1, "sector": 2, "pair": 3}  # HASHGRID_GATHER_*
+SCHEDULES = {"auto": 0, "point": 1, "level": 2}             # HASHGRID_SCHEDULE_*
 BACKWARD_MODES = {"auto": 0, "atomic": 1, "dedup": 2, "runs": 3, "dedup_adaptive": 4}  # HASHGRID_BACKWARD_*
 
 
@@ -223,7 +224,7 @@ class Resident:
     """One workload's inputs and outputs resident in HBM, plus the library handle."""
 
     def __init__(self, w: workloads.Workload, seed: int, device, backward: bool,
-                 gather: str = "auto", backward_mode: str = "auto"):
+                 gather: str = "auto", backward_mode: str = "auto", schedule: str = "auto"):
         import torch
 
         import multiresolution_hash_grid_b200 as hg
@@ -239,6 +240,7 @@ class Resident:
         self.handle = hg.hashgrid_create(w.L, w.F, w.log2T, w.N_min, w.N_max, dt)
         hg.hashgrid_set_option(self.handle, hg.HASHGRID_OPT_FORWARD_GATHER, GATHER_MODES[gather])
         hg.hashgrid_set_option(self.handle, hg.HASHGRID_OPT_BACKWARD_MODE, BACKWARD_MODES[backward_mode])
+        hg.hashgrid_set_option(self.handle, hg.HASHGRID_OPT_SCHEDULE, SCHEDULES[schedule])
         self.host = inp
 
     def forward(self, stream):
@@ -432,7 +434,7 @@ def run_b200(args) -> None:
     w = workloads.WORKLOADS[args.workload]
 
     res = Resident(w, rank_seed(rank), device, backward=w.backward, gather=args.forward_gather,
-                   backward_mode=args.backward_mode)
+                   backward_mode=args.backward_mode, schedule=args.schedule)
     sampler = ClockSampler(device.index)
     t = time_steps(res, args.steps, args.warmup, device, sampler)
     seconds = t["max_total_ms"] * 1e-3
@@ -449,7 +451,8 @@ def run_b200(args) -> None:
         "config": {"workload": w.name, "description": w.describe(), "points_per_rank": res.N,
                    "global_points": res.N * world, "parallelism": f"dp{world}: points sharded, no collective",
                    "step": "zero dL_dtable + forward + backward" if w.backward else "forward",
-                   "modes": {"forward_gather": args.forward_gather, "backward": args.backward_mode},
+                   "modes": {"forward_gather": args.forward_gather, "backward": args.backward_mode,
+                             "schedule": args.schedule},
                    "l2": "flushed before every timed step (256 MiB write, outside the events)",
                    "phase_ms": {"zero": round(t["zero_ms"], 5), "fwd": round(t["fwd_ms"], 5),
                                 "bwd": round(t["bwd_ms"], 5)}},
@@ -466,7 +469,8 @@ def run_b200(args) -> None:
 
     if not args.skip_fwd_leg and w.name != FWD_WORKLOAD:
         fw = workloads.WORKLOADS[FWD_WORKLOAD]
-        fres = Resident(fw, rank_seed(rank), device, backward=False, gather=args.forward_gather)
+        fres = Resident(fw, rank_seed(rank), device, backward=False, gather=args.forward_gather,
+                        schedule=args.schedule)
         ft = time_steps(fres, args.steps, args.warmup, device)
         fval = whole_job_rate(fres.N * args.steps, world, ft["max_total_ms"] * 1e-3)
         line["fwd"] = {"workload": fw.name, "description": fw.describe(), "value": round(fval, 1), "unit": UNIT,
@@ -503,6 +507,7 @@ def main(argv=None) -> None:
     ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--forward-gather", choices=sorted(GATHER_MODES), default="auto")
     ap.add_argument("--backward-mode", choices=sorted(BACKWARD_MODES), default="auto")
+    ap.add_argument("--schedule", choices=sorted(SCHEDULES), default="auto")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-fwd-leg", action="store_true")

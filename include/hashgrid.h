@@ -187,9 +187,29 @@ const char *hashgrid_last_error(void);
  *   HASHGRID_BACKWARD_AUTO: RUN_MERGE for F <= 4 (measured fastest on samples ordered
  *     along rays, 22% faster than ATOMIC, and within 1-14% of ATOMIC on uniformly scattered
  *     points), ATOMIC for F = 8.
+ * HASHGRID_OPT_SCHEDULE -- the order in which (point, level) pairs are visited:
+ *   HASHGRID_SCHEDULE_POINT_MAJOR: a block handles all levels of a tile of points (best
+ *     when the table fits in L2: the x and upstream-gradient rows are read once and the
+ *     output rows are written whole);
+ *   HASHGRID_SCHEDULE_LEVEL_MAJOR: blocks sweep all points for level 0, then level 1, ...,
+ *     so one level's table slice (and gradient slice) stays in L2 while every point
+ *     visits it (best for tables much larger than L2; x is read once per level). The
+ *     forward pass then gathers per corner, and the warp-dedup backward modes keep their
+ *     point-major schedule;
+ *   HASHGRID_SCHEDULE_AUTO: LEVEL_MAJOR when the table is larger than 96 MB, else
+ *     POINT_MAJOR.
  * Returns HASHGRID_ERR_ARG for an unknown option or value.
  */
-enum hashgrid_option { HASHGRID_OPT_FORWARD_GATHER = 0, HASHGRID_OPT_BACKWARD_MODE = 1 };
+enum hashgrid_option {
+    HASHGRID_OPT_FORWARD_GATHER = 0,
+    HASHGRID_OPT_BACKWARD_MODE = 1,
+    HASHGRID_OPT_SCHEDULE = 2
+};
+enum hashgrid_schedule {
+    HASHGRID_SCHEDULE_AUTO = 0,
+    HASHGRID_SCHEDULE_POINT_MAJOR = 1,
+    HASHGRID_SCHEDULE_LEVEL_MAJOR = 2
+};
 enum hashgrid_gather {
     HASHGRID_GATHER_AUTO = 0,
     HASHGRID_GATHER_CORNER = 1,

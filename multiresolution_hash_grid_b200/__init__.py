@@ -31,6 +31,10 @@ MAX_LEVELS = 32
 
 HASHGRID_OPT_FORWARD_GATHER = 0
 HASHGRID_OPT_BACKWARD_MODE = 1
+HASHGRID_OPT_SCHEDULE = 2
+HASHGRID_SCHEDULE_AUTO = 0
+HASHGRID_SCHEDULE_POINT_MAJOR = 1
+HASHGRID_SCHEDULE_LEVEL_MAJOR = 2
 HASHGRID_GATHER_AUTO = 0
 HASHGRID_GATHER_CORNER = 1
 HASHGRID_GATHER_SECTOR = 2
@@ -166,16 +170,17 @@ class HashGrid:
 
     def __init__(self, L: int = 16, F: int = 2, log2T: int = 19, N_min: int = 16, N_max: int = 512,
                  dtype: int = HASHGRID_F32, forward_gather: int = HASHGRID_GATHER_AUTO,
-                 backward_mode: int = HASHGRID_BACKWARD_AUTO):
+                 backward_mode: int = HASHGRID_BACKWARD_AUTO, schedule: int = HASHGRID_SCHEDULE_AUTO):
         self.L, self.F, self.log2T, self.N_min, self.N_max, self.dtype = L, F, log2T, N_min, N_max, dtype
         self.T = 1 << log2T
         self.handle = hashgrid_create(L, F, log2T, N_min, N_max, dtype)
         hashgrid_set_option(self.handle, HASHGRID_OPT_FORWARD_GATHER, forward_gather)
         hashgrid_set_option(self.handle, HASHGRID_OPT_BACKWARD_MODE, backward_mode)
+        hashgrid_set_option(self.handle, HASHGRID_OPT_SCHEDULE, schedule)
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h:
+        if h and lib is not None:  # the module may already be torn down at interpreter exit
             lib.hashgrid_destroy(h)
             self.handle = None
 

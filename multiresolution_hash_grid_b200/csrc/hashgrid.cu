@@ -26,6 +26,7 @@ struct hashgrid_s {
     int res[HASHGRID_MAX_LEVELS];
     int forward_gather;   // HASHGRID_GATHER_*
     int backward_mode;    // HASHGRID_BACKWARD_*
+    int schedule;         // HASHGRID_SCHEDULE_*
     hg::LevelParams lp;
 };
 
@@ -196,6 +197,40 @@ int launch_backward_mode(const hashgrid_s* h, const float* x, const float* dout,
     return launch_status("backward");
 }
 
+// Level-major when asked, or (AUTO) when the whole table is larger than most of L2.
+constexpr size_t kLevelMajorTableBytes = 96u << 20;
+
+bool level_major(const hashgrid_s* h) {
+    if (h->schedule == HASHGRID_SCHEDULE_LEVEL_MAJOR) return true;
+    if (h->schedule == HASHGRID_SCHEDULE_POINT_MAJOR) return false;
+    const size_t bytes = (size_t)h->L * ((size_t)1 << h->log2T) * h->F * (h->dtype == HASHGRID_F16 ? 2 : 4);
+    return bytes > kLevelMajorTableBytes;
+}
+
+template <int F, typename TT>
+int launch_forward_levels(const hashgrid_s* h, const float* x, int64_t N, const void* table, float* out,
+                          cudaStream_t s) {
+    const dim3 grid((unsigned)((N + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
+    hg::forward_kernel_levels<F, TT><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, N, static_cast<const TT*>(table), out);
+    return launch_status("forward");
+}
+
+template <int F>
+int launch_backward_levels(const hashgrid_s* h, const float* x, const float* dout, int64_t N, float* dtable,
+                           cudaStream_t s) {
+    if constexpr (F <= 4) {
+        if (h->backward_mode == HASHGRID_BACKWARD_RUN_MERGE || h->backward_mode == HASHGRID_BACKWARD_AUTO) {
+            const int64_t runs = (N + hg::kRun - 1) / hg::kRun;
+            const dim3 grid((unsigned)((runs + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
+            hg::backward_kernel_runs_levels<F><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, dout, N, dtable);
+            return launch_status("backward");
+        }
+    }
+    const dim3 grid((unsigned)((N + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
+    hg::backward_kernel_atomic_levels<F><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, dout, N, dtable);
+    return launch_status("backward");
+}
+
 template <int F>
 int launch_backward_runs(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
                          float* dtable, cudaStream_t s) {
@@ -210,6 +245,9 @@ int launch_backward_runs(const hashgrid_s* h, const float* x, const float* dout,
 template <int F>
 int launch_backward(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
                     float* dtable, cudaStream_t s) {
+    const bool grouped = h->backward_mode == HASHGRID_BACKWARD_WARP_DEDUP ||
+                         h->backward_mode == HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE;
+    if (!grouped && level_major(h)) return launch_backward_levels<F>(h, x, dout, N, dtable, s);
     if constexpr (F <= 4) {
         if (h->backward_mode == HASHGRID_BACKWARD_RUN_MERGE || h->backward_mode == HASHGRID_BACKWARD_AUTO)
             return launch_backward_runs<F>(h, x, dout, N, dtable, s);
@@ -286,6 +324,11 @@ int hashgrid_set_option(hashgrid_t h, int option, int value) {
                 return fail(HASHGRID_ERR_ARG, "forward gather mode %d is not a HASHGRID_GATHER_* value", value);
             h->forward_gather = value;
             return ok();
+        case HASHGRID_OPT_SCHEDULE:
+            if (value < HASHGRID_SCHEDULE_AUTO || value > HASHGRID_SCHEDULE_LEVEL_MAJOR)
+                return fail(HASHGRID_ERR_ARG, "schedule %d is not a HASHGRID_SCHEDULE_* value", value);
+            h->schedule = value;
+            return ok();
         case HASHGRID_OPT_BACKWARD_MODE:
             if (value < HASHGRID_BACKWARD_AUTO || value > HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE)
                 return fail(HASHGRID_ERR_ARG, "backward mode %d is not a HASHGRID_BACKWARD_* value", value);
@@ -304,6 +347,7 @@ int hashgrid_get_option(hashgrid_t h, int option, int* value) {
     switch (option) {
         case HASHGRID_OPT_FORWARD_GATHER: *value = h->forward_gather; return ok();
         case HASHGRID_OPT_BACKWARD_MODE: *value = h->backward_mode; return ok();
+        case HASHGRID_OPT_SCHEDULE: *value = h->schedule; return ok();
     }
     return fail(HASHGRID_ERR_ARG, "unknown option %d", option);
 }
@@ -337,6 +381,14 @@ int hashgrid_forward(hashgrid_t h, const float* x, int64_t N, const void* table,
     const int sector = h->forward_gather == HASHGRID_GATHER_SECTOR ? hg::kGatherSector
                      : h->forward_gather == HASHGRID_GATHER_PAIR   ? hg::kGatherPair
                                                                    : hg::kGatherCorner;
+    if (level_major(h)) {
+        switch (h->F) {
+            case 1: return half ? launch_forward_levels<1, __half>(h, x, N, table, out, s) : launch_forward_levels<1, float>(h, x, N, table, out, s);
+            case 2: return half ? launch_forward_levels<2, __half>(h, x, N, table, out, s) : launch_forward_levels<2, float>(h, x, N, table, out, s);
+            case 4: return half ? launch_forward_levels<4, __half>(h, x, N, table, out, s) : launch_forward_levels<4, float>(h, x, N, table, out, s);
+            case 8: return half ? launch_forward_levels<8, __half>(h, x, N, table, out, s) : launch_forward_levels<8, float>(h, x, N, table, out, s);
+        }
+    }
     switch (h->F) {
         case 1: return half ? launch_forward<1, __half>(h, x, N, table, out, sector, s) : launch_forward<1, float>(h, x, N, table, out, sector, s);
         case 2: return half ? launch_forward<2, __half>(h, x, N, table, out, sector, s) : launch_forward<2, float>(h, x, N, table, out, sector, s);

@@ -733,6 +733,63 @@ __device__ __forceinline__ void run_flush(float* dl, const float (&acc)[8][F], c
     }
 }
 
+// Walk one run of `n` consecutive points at one level (scale, mask) and reduce into the
+// level table dl. xp(j, x3) loads point j's 3 coordinates; gl(j, g) its F upstream
+// gradients.
+template <int F, class XP, class GL>
+__device__ __forceinline__ void walk_run(float* dl, float scale, uint32_t mask, int n, XP xp, GL gl) {
+    float acc[8][F];
+    uint32_t cidx[8];
+    int cv0 = 0, cv1 = 0, cv2 = 0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+#pragma unroll
+        for (int f = 0; f < F; ++f) acc[c][f] = 0.f;
+    for (int j = 0; j < n; ++j) {
+        float x3[3];
+        xp(j, x3);
+        Corners cr;
+        locate_corners(x3[0], x3[1], x3[2], scale, mask, cr);
+        float g[F];
+        gl(j, g);
+        if (j > 0) {
+            const int dx = cr.v[0] - cv0, dy = cr.v[1] - cv1, dz = cr.v[2] - cv2;
+            if ((dx | dy | dz) != 0) {
+                const bool face = abs(dx) + abs(dy) + abs(dz) == 1;
+                const int ax = face ? (dx != 0 ? 0 : (dy != 0 ? 1 : 2)) : -1;
+                const uint32_t leave_bit = (dx + dy + dz) > 0 ? 0u : 1u;
+                run_flush<F>(dl, acc, cidx, ax, leave_bit);
+                // carried corners: the new corner c with bit ax == leave_bit is the old
+                // corner c ^ (1 << ax); every other new corner starts from zero
+                float old[8][F];
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+#pragma unroll
+                    for (int f = 0; f < F; ++f) old[c][f] = acc[c][f];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const bool keep = face && (((uint32_t)c >> ax) & 1u) == leave_bit;
+#pragma unroll
+                    for (int f = 0; f < F; ++f) {
+                        const float from = ax == 0 ? old[c ^ 1][f] : (ax == 1 ? old[c ^ 2][f] : old[c ^ 4][f]);
+                        acc[c][f] = keep ? from : 0.f;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            cidx[c] = cr.idx[c];
+#pragma unroll
+            for (int f = 0; f < F; ++f) acc[c][f] = fmaf(cr.w[c], g[f], acc[c][f]);
+        }
+        cv0 = cr.v[0];
+        cv1 = cr.v[1];
+        cv2 = cr.v[2];
+    }
+    if (n > 0) run_flush<F>(dl, acc, cidx, -1, 0u);
+}
+
 template <int F>
 __global__ void __launch_bounds__(256) backward_kernel_runs(LevelParams lp, const float* __restrict__ x,
                                                            const float* __restrict__ dout, int64_t N,
@@ -778,56 +835,163 @@ __global__ void __launch_bounds__(256) backward_kernel_runs(LevelParams lp, cons
     const int jmax = min(kRun, nvalid - lane * kRun);  // points of this lane's run (may be <= 0)
     for (int l = warp; l < L; l += nwarps) {
         float* dl = dtable + (uint64_t)l * lp.T * F;
-        float acc[8][F];
-        uint32_t cidx[8];
-        int cv0 = 0, cv1 = 0, cv2 = 0;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-#pragma unroll
-            for (int f = 0; f < F; ++f) acc[c][f] = 0.f;
-        for (int j = 0; j < jmax; ++j) {
-            const float* xp = xs + lane * XS + j * 3;
-            Corners cr;
-            locate_corners(xp[0], xp[1], xp[2], lp.scale[l], lp.mask, cr);
-            float g[F];
-            load_smem_entry<F>(gs + lane * G + j * S + l * F, g);
-            if (j > 0) {
-                const int dx = cr.v[0] - cv0, dy = cr.v[1] - cv1, dz = cr.v[2] - cv2;
-                if ((dx | dy | dz) != 0) {
-                    const bool face = abs(dx) + abs(dy) + abs(dz) == 1;
-                    const int ax = face ? (dx != 0 ? 0 : (dy != 0 ? 1 : 2)) : -1;
-                    const uint32_t leave_bit = (dx + dy + dz) > 0 ? 0u : 1u;
-                    run_flush<F>(dl, acc, cidx, ax, leave_bit);
-                    // carried corners: the new corner c with bit ax == leave_bit is the old
-                    // corner c ^ (1 << ax); every other new corner starts from zero
-                    float old[8][F];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-#pragma unroll
-                        for (int f = 0; f < F; ++f) old[c][f] = acc[c][f];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const bool keep = face && (((uint32_t)c >> ax) & 1u) == leave_bit;
-#pragma unroll
-                        for (int f = 0; f < F; ++f) {
-                            const float from = ax == 0 ? old[c ^ 1][f] : (ax == 1 ? old[c ^ 2][f] : old[c ^ 4][f]);
-                            acc[c][f] = keep ? from : 0.f;
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                cidx[c] = cr.idx[c];
-#pragma unroll
-                for (int f = 0; f < F; ++f) acc[c][f] = fmaf(cr.w[c], g[f], acc[c][f]);
-            }
-            cv0 = cr.v[0];
-            cv1 = cr.v[1];
-            cv2 = cr.v[2];
-        }
-        if (jmax > 0) run_flush<F>(dl, acc, cidx, -1, 0u);
+        walk_run<F>(dl, lp.scale[l], lp.mask, jmax,
+                    [&](int j, float* x3) {
+                        const float* q = xs + lane * XS + j * 3;
+                        x3[0] = q[0]; x3[1] = q[1]; x3[2] = q[2];
+                    },
+                    [&](int j, float* g) { load_smem_entry<F>(gs + lane * G + j * S + l * F, g); });
     }
+}
+
+// ---------------------------------------------------------------------------------------
+// Level-major schedules, for tables larger than L2. Grid (tiles, L): blocks are issued with
+// the tile index fastest, so the GPU works through the levels one after another and the
+// current level's table slice (backward: its gradient slice) stays resident in L2 while
+// every point visits it, instead of each point's fine-level gathers missing to DRAM. The
+// price is re-reading x once per level and touching output / upstream-gradient rows in
+// F-wide column slices.
+// ---------------------------------------------------------------------------------------
+// Streaming (evict-first) row accesses: x, output and upstream-gradient slices are touched
+// once per level and must not push the level's table out of L2.
+template <int F>
+__device__ __forceinline__ void store_global_entry(float* p, const float* v) {
+    if constexpr (F == 1) {
+        __stcs(p, v[0]);
+    } else if constexpr (F == 2) {
+        __stcs(reinterpret_cast<float2*>(p), make_float2(v[0], v[1]));
+    } else {
+#pragma unroll
+        for (int j = 0; j < F; j += 4)
+            __stcs(reinterpret_cast<float4*>(p + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+    }
+}
+
+template <int F>
+__device__ __forceinline__ void load_global_entry(const float* p, float* v) {
+    if constexpr (F == 1) {
+        v[0] = __ldcs(p);
+    } else if constexpr (F == 2) {
+        float2 a = __ldcs(reinterpret_cast<const float2*>(p));
+        v[0] = a.x; v[1] = a.y;
+    } else {
+#pragma unroll
+        for (int j = 0; j < F; j += 4) {
+            float4 a = __ldcs(reinterpret_cast<const float4*>(p + j));
+            v[j] = a.x; v[j + 1] = a.y; v[j + 2] = a.z; v[j + 3] = a.w;
+        }
+    }
+}
+
+// L2 policy that keeps lines resident (evict-last), for the level's table slice.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// F-wide fp32 / fp16 table entry load with an L2 cache policy.
+template <int F, typename TT>
+__device__ __forceinline__ void load_entry_policy(const TT* p, float* e, uint64_t pol) {
+    constexpr int E = F * (int)sizeof(TT);
+    uint32_t w[8];
+    if constexpr (E == 2) {
+        unsigned short h;
+        asm("ld.global.nc.L2::cache_hint.b16 %0, [%1], %2;" : "=h"(h) : "l"(p), "l"(pol));
+        e[0] = __half2float(__ushort_as_half(h));
+        return;
+    } else if constexpr (E == 4) {
+        asm("ld.global.nc.L2::cache_hint.b32 %0, [%1], %2;" : "=r"(w[0]) : "l"(p), "l"(pol));
+    } else if constexpr (E == 8) {
+        asm("ld.global.nc.L2::cache_hint.v2.b32 {%0, %1}, [%2], %3;" : "=r"(w[0]), "=r"(w[1]) : "l"(p), "l"(pol));
+    } else {
+#pragma unroll
+        for (int k = 0; k < E / 16; ++k)
+            asm("ld.global.nc.L2::cache_hint.v4.b32 {%0, %1, %2, %3}, [%4], %5;"
+                : "=r"(w[4 * k]), "=r"(w[4 * k + 1]), "=r"(w[4 * k + 2]), "=r"(w[4 * k + 3])
+                : "l"(reinterpret_cast<const char*>(p) + 16 * k), "l"(pol));
+    }
+    if constexpr (sizeof(TT) == 4) {
+#pragma unroll
+        for (int f = 0; f < F; ++f) e[f] = __uint_as_float(w[f]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < E / 4; ++k) {
+            float2 v = h2_bits_to_f2(w[k]);
+            e[2 * k] = v.x;
+            e[2 * k + 1] = v.y;
+        }
+    }
+}
+
+constexpr int kLevelBlock = 256;
+
+template <int F, typename TT>
+__global__ void __launch_bounds__(kLevelBlock) forward_kernel_levels(LevelParams lp, const float* __restrict__ x,
+                                                                    int64_t N, const TT* __restrict__ table,
+                                                                    float* __restrict__ out) {
+    const int l = blockIdx.y;
+    const int64_t p = (int64_t)blockIdx.x * kLevelBlock + threadIdx.x;
+    if (p >= N) return;
+    Corners cr;
+    locate_corners(__ldcs(x + p * 3), __ldcs(x + p * 3 + 1), __ldcs(x + p * 3 + 2), lp.scale[l], lp.mask, cr);
+    const TT* tl = table + (uint64_t)l * lp.T * F;
+    const uint64_t pol = l2_evict_last_policy();
+    float e[8][F];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) load_entry_policy<F, TT>(tl + (uint64_t)cr.idx[c] * F, e[c], pol);
+    float o[F];
+#pragma unroll
+    for (int f = 0; f < F; ++f) {
+        float acc = cr.w[0] * e[0][f];
+#pragma unroll
+        for (int c = 1; c < 8; ++c) acc = fmaf(cr.w[c], e[c][f], acc);
+        o[f] = acc;
+    }
+    store_global_entry<F>(out + p * (int64_t)(lp.L * F) + l * F, o);
+}
+
+template <int F>
+__global__ void __launch_bounds__(kLevelBlock) backward_kernel_atomic_levels(LevelParams lp, const float* __restrict__ x,
+                                                                            const float* __restrict__ dout, int64_t N,
+                                                                            float* __restrict__ dtable) {
+    const int l = blockIdx.y;
+    const int64_t p = (int64_t)blockIdx.x * kLevelBlock + threadIdx.x;
+    if (p >= N) return;
+    Corners cr;
+    locate_corners(__ldcs(x + p * 3), __ldcs(x + p * 3 + 1), __ldcs(x + p * 3 + 2), lp.scale[l], lp.mask, cr);
+    float g[F];
+    load_global_entry<F>(dout + p * (int64_t)(lp.L * F) + l * F, g);
+    float* dl = dtable + (uint64_t)l * lp.T * F;
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+        float va[F], vb[F];
+#pragma unroll
+        for (int f = 0; f < F; ++f) {
+            va[f] = cr.w[2 * qq] * g[f];
+            vb[f] = cr.w[2 * qq + 1] * g[f];
+        }
+        red_pair<F>(dl, cr.idx[2 * qq], cr.idx[2 * qq + 1], va, vb);
+    }
+}
+
+// One thread walks one run of kRun consecutive points at level blockIdx.y.
+template <int F>
+__global__ void __launch_bounds__(kLevelBlock) backward_kernel_runs_levels(LevelParams lp, const float* __restrict__ x,
+                                                                          const float* __restrict__ dout, int64_t N,
+                                                                          float* __restrict__ dtable) {
+    const int l = blockIdx.y;
+    const int64_t p0 = ((int64_t)blockIdx.x * kLevelBlock + threadIdx.x) * kRun;
+    if (p0 >= N) return;
+    const int n = (int)min((int64_t)kRun, N - p0);
+    const int64_t W = lp.L * F;
+    float* dl = dtable + (uint64_t)l * lp.T * F;
+    walk_run<F>(dl, lp.scale[l], lp.mask, n,
+                [&](int j, float* x3) {
+                    const float* q = x + (p0 + j) * 3;
+                    x3[0] = __ldcs(q); x3[1] = __ldcs(q + 1); x3[2] = __ldcs(q + 2);
+                },
+                [&](int j, float* g) { load_global_entry<F>(dout + (p0 + j) * W + l * F, g); });
 }
 
 // ---------------------------------------------------------------------------------------

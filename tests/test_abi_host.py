@@ -106,7 +106,10 @@ def test_options():
         hg.hashgrid_set_option(h, hg.HASHGRID_OPT_BACKWARD_MODE, hg.HASHGRID_BACKWARD_WARP_DEDUP)
         assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_FORWARD_GATHER) == hg.HASHGRID_GATHER_SECTOR
         assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_BACKWARD_MODE) == hg.HASHGRID_BACKWARD_WARP_DEDUP
-        for opt, val in [(hg.HASHGRID_OPT_FORWARD_GATHER, 4), (hg.HASHGRID_OPT_BACKWARD_MODE, -1), (hg.HASHGRID_OPT_BACKWARD_MODE, 5), (7, 0)]:
+        assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_SCHEDULE) == hg.HASHGRID_SCHEDULE_AUTO
+        hg.hashgrid_set_option(h, hg.HASHGRID_OPT_SCHEDULE, hg.HASHGRID_SCHEDULE_LEVEL_MAJOR)
+        assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_SCHEDULE) == hg.HASHGRID_SCHEDULE_LEVEL_MAJOR
+        for opt, val in [(hg.HASHGRID_OPT_SCHEDULE, 3), (hg.HASHGRID_OPT_FORWARD_GATHER, 4), (hg.HASHGRID_OPT_BACKWARD_MODE, -1), (hg.HASHGRID_OPT_BACKWARD_MODE, 5), (7, 0)]:
             assert hg.lib.hashgrid_set_option(h, opt, val) == hg.HASHGRID_ERR_ARG
         assert hg.lib.hashgrid_set_option(None, 0, 0) == hg.HASHGRID_ERR_ARG
     finally:

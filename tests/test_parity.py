@@ -44,7 +44,7 @@ GATHERS = ["corner", "sector", "pair"]
 BACKWARDS = ["atomic", "auto", "dedup", "runs", "dedup_adaptive"]
 
 
-def make_pair(L, F, log2T, N_min, N_max, dtype="f32", gather="auto", backward="auto"):
+def make_pair(L, F, log2T, N_min, N_max, dtype="f32", gather="auto", backward="auto", schedule="auto"):
     hg = hgmod()
     dt = hg.HASHGRID_F16 if dtype == "f16" else hg.HASHGRID_F32
     gm = {"auto": hg.HASHGRID_GATHER_AUTO, "corner": hg.HASHGRID_GATHER_CORNER,
@@ -53,7 +53,9 @@ def make_pair(L, F, log2T, N_min, N_max, dtype="f32", gather="auto", backward="a
           "dedup": hg.HASHGRID_BACKWARD_WARP_DEDUP if F <= 4 else hg.HASHGRID_BACKWARD_ATOMIC,
           "runs": hg.HASHGRID_BACKWARD_RUN_MERGE if F <= 4 else hg.HASHGRID_BACKWARD_ATOMIC,
           "dedup_adaptive": hg.HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE if F <= 4 else hg.HASHGRID_BACKWARD_ATOMIC}[backward]
-    return (hg.HashGrid(L, F, log2T, N_min, N_max, dt, forward_gather=gm, backward_mode=bm),
+    sm = {"auto": hg.HASHGRID_SCHEDULE_AUTO, "point": hg.HASHGRID_SCHEDULE_POINT_MAJOR,
+          "level": hg.HASHGRID_SCHEDULE_LEVEL_MAJOR}[schedule]
+    return (hg.HashGrid(L, F, log2T, N_min, N_max, dt, forward_gather=gm, backward_mode=bm, schedule=sm),
             oracle.Grid(L, F, log2T, N_min, N_max, oracle.F16 if dtype == "f16" else oracle.F32))
 
 
@@ -120,20 +122,24 @@ def test_indices_bit_exact(name, reduced_inputs):
     np.testing.assert_array_equal(got, want)
 
 
-@pytest.mark.parametrize("gather", GATHERS)
+@pytest.mark.parametrize("gather", GATHERS + ["level"])
 @pytest.mark.parametrize("name", list(workloads.WORKLOADS))
 def test_forward_parity(name, gather, reduced_inputs):
     w, inp = reduced_inputs(name)
-    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, gather=gather)
+    if gather == "level":
+        grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, schedule="level")
+    else:
+        grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, gather=gather, schedule="point")
     got = gpu_forward(grid, inp.x, inp.table)
     check_forward(og, inp.x, inp.table, got, w.dtype)
 
 
-@pytest.mark.parametrize("mode", BACKWARDS)
+@pytest.mark.parametrize("mode", BACKWARDS + ["runs/level", "atomic/level"])
 @pytest.mark.parametrize("name", list(workloads.WORKLOADS))
 def test_backward_parity(name, mode, reduced_inputs):
     w, inp = reduced_inputs(name)
-    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, backward=mode)
+    bm, _, sched = mode.partition("/")
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, backward=bm, schedule=sched or "point")
     got = gpu_backward(grid, inp.x, inp.g)
     ref = og.backward(inp.x, inp.g, nthreads=THREADS)
     assert rel_l2(got, ref) <= BWD_REL_L2
@@ -153,12 +159,13 @@ FULL_LEVELS = {   # gradient levels the oracle recomputes at full size (bounded 
 }
 
 
-@pytest.mark.parametrize("modes", [("auto", "auto"), ("corner", "dedup"), ("sector", "runs")])
+@pytest.mark.parametrize("modes", [("auto", "auto", "auto"), ("corner", "dedup", "point"), ("sector", "runs", "point"),
+                                   ("auto", "auto", "level")])
 @pytest.mark.parametrize("name", list(workloads.WORKLOADS))
 def test_full_size(name, modes):
     w = workloads.WORKLOADS[name]
     inp = workloads.make_inputs(w, seed=0, grads=True)
-    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, gather=modes[0], backward=modes[1])
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, gather=modes[0], backward=modes[1], schedule=modes[2])
     x_d, t_d, g_d = dev(inp.x), dev(inp.table), dev(inp.g)
     out_d = grid.forward(x_d, t_d)
     dt_d = grid.backward(x_d, g_d)
@@ -187,10 +194,11 @@ def test_full_size(name, modes):
 # Edge cases
 # ---------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto"), ("pair", "runs")])
+@pytest.mark.parametrize("modes", [("corner", "atomic", "point"), ("sector", "dedup", "point"), ("auto", "auto", "point"),
+                                   ("pair", "runs", "point"), ("auto", "auto", "level"), ("auto", "atomic", "level")])
 @pytest.mark.parametrize("N", [1, 2, 31, 32, 33, 63, 64, 65, 127, 129, 1000])
 def test_ragged_batch_sizes(N, modes):
-    grid, og = make_pair(16, 2, 19, 16, 512, gather=modes[0], backward=modes[1])
+    grid, og = make_pair(16, 2, 19, 16, 512, gather=modes[0], backward=modes[1], schedule=modes[2])
     rng = np.random.default_rng(N)
     table = workloads.table_values(rng, 16, 2**19, 2)
     x = workloads.uniform_points(rng, N)
@@ -199,11 +207,12 @@ def test_ragged_batch_sizes(N, modes):
     assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g, nthreads=THREADS)) <= BWD_REL_L2
 
 
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto"), ("pair", "runs")])
+@pytest.mark.parametrize("modes", [("corner", "atomic", "point"), ("sector", "dedup", "point"), ("auto", "auto", "point"),
+                                   ("pair", "runs", "point"), ("auto", "auto", "level"), ("auto", "atomic", "level")])
 def test_special_coordinates(modes):
     """x = 0, the largest fp32 below 1, exactly 1 (voxel N_l, corner N_l + 1), points
     outside the cube (no clamping), and grid vertices (bit-exact table entries)."""
-    grid, og = make_pair(4, 2, 10, 2, 16, gather=modes[0], backward=modes[1])
+    grid, og = make_pair(4, 2, 10, 2, 16, gather=modes[0], backward=modes[1], schedule=modes[2])
     rng = np.random.default_rng(5)
     table = rng.standard_normal((4, 1024, 2)).astype(np.float32)
     vals = np.array([0.0, 1.0 - 2**-24, 1.0, 0.5, 0.25, -0.3, 1.7, -2.0, 3.25], dtype=np.float32)
@@ -219,11 +228,12 @@ def test_special_coordinates(modes):
     assert rel_l2(gpu_backward(grid, x, g), og.backward(x, g)) <= BWD_REL_L2
 
 
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto"), ("pair", "runs")])
+@pytest.mark.parametrize("modes", [("corner", "atomic", "point"), ("sector", "dedup", "point"), ("auto", "auto", "point"),
+                                   ("pair", "runs", "point"), ("auto", "auto", "level"), ("auto", "atomic", "level")])
 @pytest.mark.parametrize("F", [1, 2, 4, 8])
 @pytest.mark.parametrize("dtype", ["f32", "f16"])
 def test_feature_widths_and_dtypes(F, dtype, modes):
-    grid, og = make_pair(5, F, 12, 3, 200, dtype, gather=modes[0], backward=modes[1])
+    grid, og = make_pair(5, F, 12, 3, 200, dtype, gather=modes[0], backward=modes[1], schedule=modes[2])
     rng = np.random.default_rng(F)
     table = workloads.table_values(rng, 5, 2**12, F, dtype)
     x = workloads.uniform_points(rng, 3000)
@@ -239,10 +249,11 @@ def test_feature_widths_and_dtypes(F, dtype, modes):
     (2, 1, 24, 512, 2**16),      # largest table
     (32, 8, 8, 2, 300),          # widest output row (256 floats, > 48 KB of shared memory)
 ])
-@pytest.mark.parametrize("modes", [("corner", "atomic"), ("sector", "dedup"), ("auto", "auto"), ("pair", "runs")])
+@pytest.mark.parametrize("modes", [("corner", "atomic", "point"), ("sector", "dedup", "point"), ("auto", "auto", "point"),
+                                   ("pair", "runs", "point"), ("auto", "auto", "level"), ("auto", "atomic", "level")])
 def test_extreme_shapes(shape, modes):
     L, F, log2T, a, b = shape
-    grid, og = make_pair(L, F, log2T, a, b, gather=modes[0], backward=modes[1])
+    grid, og = make_pair(L, F, log2T, a, b, gather=modes[0], backward=modes[1], schedule=modes[2])
     rng = np.random.default_rng(L * 100 + F)
     table = workloads.table_values(rng, L, 2**log2T, F)
     x = workloads.uniform_points(rng, 777)
