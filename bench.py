@@ -309,36 +309,60 @@ def time_steps(res: Resident, steps: int, warmup: int, device, sampler=None) -> 
 
 def time_e2e(res: Resident, steps: int, warmup: int, device) -> dict:
     """End to end through the C ABI from pinned host buffers: per step, copy x (and the
-    upstream gradient) host->device, forward (+ zero + backward), copy the encoding back to
-    pinned host memory. The gradient table stays on the device for the optimizer."""
+    upstream gradient) host->device, zero the gradient, forward, backward, and copy the
+    encoding back to pinned host memory. The gradient table stays on the device for the
+    optimizer. Steps are pipelined on three streams with double buffers: the upload of
+    step k+1 and the download of step k-1 overlap step k's kernels (PCIe is full duplex)."""
     import torch
-    stream = torch.cuda.current_stream(device)
-    sp = stream.cuda_stream
+    hg = res.hg
+    s_in, s_comp, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device), torch.cuda.Stream(device)
     xh = torch.from_numpy(res.host.x).pin_memory()
     gh = torch.from_numpy(res.host.g).pin_memory() if res.backward else None
-    oh = torch.empty(res.out.shape, dtype=torch.float32).pin_memory()
+    xd = [res.x, torch.empty_like(res.x)]
+    gd = [res.g, torch.empty_like(res.g)] if res.backward else [None, None]
+    od = [res.out, torch.empty_like(res.out)]
+    oh = [torch.empty(res.out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = xh.numel() * 4 + (gh.numel() * 4 if gh is not None else 0)
-    d2h = oh.numel() * 4
+    d2h = oh[0].numel() * 4
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for b in range(2):   # every buffer starts free
+        ev_comp[b].record(s_comp)
+        ev_out[b].record(s_out)
 
-    def one():
-        res.x.copy_(xh, non_blocking=True)
-        if gh is not None:
-            res.g.copy_(gh, non_blocking=True)
-            res.dtable.zero_()
-        res.forward(sp)
-        if res.backward:
-            res.backward_pass(sp)
-        oh.copy_(res.out, non_blocking=True)
+    def one(k):
+        b = k % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_comp[b])              # step k-2 no longer reads xd[b], gd[b]
+            xd[b].copy_(xh, non_blocking=True)
+            if gh is not None:
+                gd[b].copy_(gh, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[b])
+            s_comp.wait_event(ev_out[b])             # step k-2's download of od[b] is done
+            sp = s_comp.cuda_stream
+            if res.backward:
+                res.dtable.zero_()
+            hg.hashgrid_forward(res.handle, xd[b], res.N, res.table, od[b], sp)
+            if res.backward:
+                hg.hashgrid_backward(res.handle, xd[b], gd[b], res.N, res.dtable, sp)
+            ev_comp[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            oh[b].copy_(od[b], non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(warmup):
-        one()
+    for k in range(warmup):
+        one(k)
     torch.cuda.synchronize(device)
     barrier(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
+    e0.record(s_in)
+    for k in range(steps):
+        one(warmup + k)
+    e1.record(s_out)
     torch.cuda.synchronize(device)
     ms = max_over_ranks(e0.elapsed_time(e1), device)
     return {"ms": ms, "h2d": h2d, "d2h": d2h}
@@ -482,6 +506,7 @@ def run_b200(args) -> None:
 
     if not args.skip_e2e:
         e = time_e2e(res, args.steps, min(args.warmup, 3), device)
+        launches += args.steps * (2 if w.backward else 1)
         line["e2e"] = {"value": round(res.N * world * args.steps / (e["ms"] * 1e-3), 1), "unit": UNIT,
                        "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                        "note": "pinned host x (and upstream grads) -> device, zero + fwd + bwd through "

@@ -140,6 +140,47 @@ int hashgrid_backward(hashgrid_t h, const float *x, const float *dL_dout, int64_
                       float *dL_dtable, void *cuda_stream);
 
 /*
+ * hashgrid_backward_input -- gradient of a loss with respect to the input coordinates.
+ *
+ * [NeRFace-HG] section 3 applies the encoder to coordinates produced by a learned
+ * transform, which needs dL/dx. Inside the voxel that floor() selects,
+ * d frac_i / d x_i = N_l, so
+ *   dL_dx[p][i] = sum_l N_l * sum_c (sum_f dL_dout[p][l*F + f] * table[l][index_c][f])
+ *                 * (offset_i(c) ? +1 : -1) * prod_{j != i} (offset_j(c) ? frac_j : 1 - frac_j).
+ * On a voxel face the encoding has a kink; this is the derivative from the voxel that
+ * contains x (the one-sided derivative towards +x). fp32 arithmetic, levels summed in order.
+ *
+ * x: [N,3] fp32; dL_dout: [N,L*F] fp32; table: [L,T,F] of the handle's dtype;
+ * dL_dx: [N,3] fp32, OVERWRITTEN. Always point-major (schedule option ignored).
+ */
+int hashgrid_backward_input(hashgrid_t h, const float *x, const float *dL_dout, int64_t N,
+                            const void *table, float *dL_dx, void *cuda_stream);
+
+/*
+ * hashgrid_adam_step -- one sparse Adam step on the tables, fused with clearing the
+ * consumed gradient.
+ *
+ * [NeRFace-HG] sections 3 and 4: the tables are trained with Adam, without weight decay,
+ * at a learning rate several times the MLP's, and only the sampled entries receive
+ * gradient in a step; [Overview-HG] sections 4-5 use Adam with lr 1e-2 .. 1e-3. For every
+ * element (L*T*F of them) with a nonzero gradient g, at step t >= 1:
+ *   m = beta1 m + (1 - beta1) g;   v = beta2 v + (1 - beta2) g^2;
+ *   table -= lr * (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps);
+ * elements whose gradient is exactly zero were not sampled and are left unchanged (table,
+ * m and v). fp32 arithmetic with correctly rounded sqrt and division; fp16 tables are
+ * updated in fp32 and stored rounded to nearest. If zero_grad != 0 the consumed gradient
+ * elements are set to zero, so dL_dtable is all zeros afterwards and the next backward can
+ * accumulate into it without a separate clear.
+ *
+ * table: [L,T,F] of the handle's dtype (updated); adam_m, adam_v: [L,T,F] fp32 moments
+ * (updated; zero them before step 1); dL_dtable: [L,T,F] fp32. step >= 1,
+ * 0 <= beta1, beta2 < 1, eps > 0, lr finite; otherwise HASHGRID_ERR_ARG.
+ */
+int hashgrid_adam_step(hashgrid_t h, void *table, float *adam_m, float *adam_v, float *dL_dtable,
+                       int64_t step, float lr, float beta1, float beta2, float eps, int zero_grad,
+                       void *cuda_stream);
+
+/*
  * hashgrid_debug_indices -- export the hash index of every corner: idx_out[(p*L + l)*8 + c]
  * = index_c of point p at level l (uint32, < T), computed by the same device code as the
  * forward and backward passes. For tests and inspection. idx_out: [N, L, 8] uint32.

@@ -68,6 +68,9 @@ def _load() -> ctypes.CDLL:
         "hashgrid_get_option": (i32, [vp, i32, ctypes.POINTER(i32)]),
         "hashgrid_forward": (i32, [vp, vp, i64, vp, vp, vp]),
         "hashgrid_backward": (i32, [vp, vp, vp, i64, vp, vp]),
+        "hashgrid_backward_input": (i32, [vp, vp, vp, i64, vp, vp, vp]),
+        "hashgrid_adam_step": (i32, [vp, vp, vp, vp, vp, i64, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                     ctypes.c_float, i32, vp]),
         "hashgrid_debug_indices": (i32, [vp, vp, i64, vp, vp]),
         "hashgrid_last_error": (ctypes.c_char_p, []),
         "hashgrid_version": (ctypes.c_char_p, []),
@@ -159,6 +162,16 @@ def hashgrid_backward(h: int, x, dL_dout, N: int, dL_dtable, stream=None) -> Non
     _check(lib.hashgrid_backward(h, _ptr(x), _ptr(dL_dout), N, _ptr(dL_dtable), _stream(stream)))
 
 
+def hashgrid_backward_input(h: int, x, dL_dout, N: int, table, dL_dx, stream=None) -> None:
+    _check(lib.hashgrid_backward_input(h, _ptr(x), _ptr(dL_dout), N, _ptr(table), _ptr(dL_dx), _stream(stream)))
+
+
+def hashgrid_adam_step(h: int, table, adam_m, adam_v, dL_dtable, step: int, lr: float, beta1: float = 0.9,
+                       beta2: float = 0.99, eps: float = 1e-15, zero_grad: bool = True, stream=None) -> None:
+    _check(lib.hashgrid_adam_step(h, _ptr(table), _ptr(adam_m), _ptr(adam_v), _ptr(dL_dtable), step, lr, beta1,
+                                  beta2, eps, 1 if zero_grad else 0, _stream(stream)))
+
+
 def hashgrid_debug_indices(h: int, x, N: int, idx_out, stream=None) -> None:
     _check(lib.hashgrid_debug_indices(h, _ptr(x), N, _ptr(idx_out), _stream(stream)))
 
@@ -202,6 +215,13 @@ class HashGrid:
             dL_dtable = torch.zeros((self.L, self.T, self.F), dtype=torch.float32, device=x.device)
         hashgrid_backward(self.handle, x, dL_dout, x.shape[0], dL_dtable, stream)
         return dL_dtable
+
+    def backward_input(self, x, dL_dout, table, dL_dx=None, stream=None):
+        import torch
+        if dL_dx is None:
+            dL_dx = torch.empty((x.shape[0], 3), dtype=torch.float32, device=x.device)
+        hashgrid_backward_input(self.handle, x, dL_dout, x.shape[0], table, dL_dx, stream)
+        return dL_dx
 
     def indices(self, x, stream=None):
         import torch

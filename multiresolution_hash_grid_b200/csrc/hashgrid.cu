@@ -259,6 +259,17 @@ int launch_backward(const hashgrid_s* h, const float* x, const float* dout, int6
     return launch_backward_mode<F, hg::kAtomicOnly>(h, x, dout, N, dtable, s);
 }
 
+template <int F, typename TT>
+int launch_backward_input(const hashgrid_s* h, const float* x, const float* dout, int64_t N, const void* table,
+                          float* dx, cudaStream_t s) {
+    auto k = hg::backward_input_kernel<F, TT, kTile>;
+    const size_t smem = hg::input_grad_smem_bytes(kTile, h->L, F);
+    if (int rc = prepare_smem(k, smem)) return rc;
+    const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
+    k<<<blocks, tile_threads(h->L), smem, s>>>(h->lp, x, dout, N, static_cast<const TT*>(table), dx);
+    return launch_status("backward_input");
+}
+
 size_t table_bytes(const hashgrid_s* h) {
     return (size_t)h->L * ((size_t)1 << h->log2T) * (size_t)h->F * (h->dtype == HASHGRID_F16 ? 2 : 4);
 }
@@ -415,6 +426,61 @@ int hashgrid_backward(hashgrid_t h, const float* x, const float* dL_dout, int64_
         case 8: return launch_backward<8>(h, x, dL_dout, N, dL_dtable, s);
     }
     return fail(HASHGRID_ERR_ARG, "corrupt handle");
+}
+
+int hashgrid_backward_input(hashgrid_t h, const float* x, const float* dL_dout, int64_t N, const void* table,
+                            float* dL_dx, void* cuda_stream) {
+    if (int rc = check_handle(h)) return rc;
+    if (int rc = check_N(N, kTile)) return rc;
+    if (N == 0) return ok();
+    const size_t W = (size_t)h->L * h->F;
+    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(dL_dout, (size_t)N * W * sizeof(float), "dL_dout")) return rc;
+    if (int rc = check_buffer(table, table_bytes(h), "table")) return rc;
+    if (int rc = check_buffer(dL_dx, (size_t)N * 3 * sizeof(float), "dL_dx")) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    const bool half = h->dtype == HASHGRID_F16;
+    switch (h->F) {
+        case 1: return half ? launch_backward_input<1, __half>(h, x, dL_dout, N, table, dL_dx, s) : launch_backward_input<1, float>(h, x, dL_dout, N, table, dL_dx, s);
+        case 2: return half ? launch_backward_input<2, __half>(h, x, dL_dout, N, table, dL_dx, s) : launch_backward_input<2, float>(h, x, dL_dout, N, table, dL_dx, s);
+        case 4: return half ? launch_backward_input<4, __half>(h, x, dL_dout, N, table, dL_dx, s) : launch_backward_input<4, float>(h, x, dL_dout, N, table, dL_dx, s);
+        case 8: return half ? launch_backward_input<8, __half>(h, x, dL_dout, N, table, dL_dx, s) : launch_backward_input<8, float>(h, x, dL_dout, N, table, dL_dx, s);
+    }
+    return fail(HASHGRID_ERR_ARG, "corrupt handle");
+}
+
+int hashgrid_adam_step(hashgrid_t h, void* table, float* adam_m, float* adam_v, float* dL_dtable, int64_t step,
+                       float lr, float beta1, float beta2, float eps, int zero_grad, void* cuda_stream) {
+    if (int rc = check_handle(h)) return rc;
+    if (step < 1) return fail(HASHGRID_ERR_ARG, "step = %lld must be >= 1", (long long)step);
+    if (!(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
+        return fail(HASHGRID_ERR_ARG, "betas (%g, %g) must lie in [0, 1)", beta1, beta2);
+    if (!(eps > 0.f) || !std::isfinite(eps) || !std::isfinite(lr))
+        return fail(HASHGRID_ERR_ARG, "lr = %g and eps = %g must be finite, eps > 0", lr, eps);
+    const size_t n = hashgrid_table_elems(h);
+    if (int rc = check_buffer(table, table_bytes(h), "table")) return rc;
+    if (int rc = check_buffer(adam_m, n * sizeof(float), "adam_m")) return rc;
+    if (int rc = check_buffer(adam_v, n * sizeof(float), "adam_v")) return rc;
+    if (int rc = check_buffer(dL_dtable, n * sizeof(float), "dL_dtable")) return rc;
+    hg::AdamParams a;
+    a.lr = lr;
+    a.b1 = beta1;
+    a.b2 = beta2;
+    a.eps = eps;
+    a.c1 = (float)(1.0 / (1.0 - std::pow((double)beta1, (double)step)));
+    a.c2 = (float)(1.0 / (1.0 - std::pow((double)beta2, (double)step)));
+    const int64_t n4 = (int64_t)(n / 4);  // L*T*F is a multiple of 16
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (n4 + 255) / 256;
+    const unsigned blocks = (unsigned)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    if (h->dtype == HASHGRID_F16)
+        hg::adam_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<__half*>(table), adam_m, adam_v, dL_dtable, n4, a, zero_grad);
+    else
+        hg::adam_kernel<float><<<blocks, 256, 0, s>>>(static_cast<float*>(table), adam_m, adam_v, dL_dtable, n4, a, zero_grad);
+    return launch_status("adam_step");
 }
 
 int hashgrid_debug_indices(hashgrid_t h, const float* x, int64_t N, uint32_t* idx_out, void* cuda_stream) {

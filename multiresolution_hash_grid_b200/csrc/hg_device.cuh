@@ -240,6 +240,7 @@ struct Corners {
     uint32_t idx[8];
     float w[8];
     int v[3];  // the voxel (lower corner)
+    float f[3];  // position inside the voxel
 };
 
 __device__ __forceinline__ void locate_corners(float x0, float x1, float x2, float scale,
@@ -256,6 +257,9 @@ __device__ __forceinline__ void locate_corners(float x0, float x1, float x2, flo
     const float f0 = __fsub_rn(xs0, __int2float_rn(v0));
     const float f1 = __fsub_rn(xs1, __int2float_rn(v1));
     const float f2 = __fsub_rn(xs2, __int2float_rn(v2));
+    cr.f[0] = f0;
+    cr.f[1] = f1;
+    cr.f[2] = f2;
     const uint32_t hx0 = (uint32_t)v0, hx1 = hx0 + 1u;
     const uint32_t hy0 = (uint32_t)v1 * kPrimeY, hy1 = hy0 + kPrimeY;
     const uint32_t hz0 = (uint32_t)v2 * kPrimeZ, hz1 = hz0 + kPrimeZ;
@@ -992,6 +996,149 @@ __global__ void __launch_bounds__(kLevelBlock) backward_kernel_runs_levels(Level
                     x3[0] = __ldcs(q); x3[1] = __ldcs(q + 1); x3[2] = __ldcs(q + 2);
                 },
                 [&](int j, float* g) { load_global_entry<F>(dout + (p0 + j) * W + l * F, g); });
+}
+
+// ---------------------------------------------------------------------------------------
+// Gradient with respect to the input coordinates ([NeRFace-HG] section 3 runs the encoder
+// on coordinates produced by a learned transform). Inside the voxel that floor() selects,
+// d frac_i / d x_i = N_l, so with s_c = sum_f g_f e_c[f]:
+//   dL/dx_i = sum_l N_l * sum_c s_c * (d_i ? +1 : -1) * prod_{j != i} (d_j ? frac_j : 1 - frac_j).
+// Point-major: a block stages its x and upstream-gradient rows, each (point, level) thread
+// gathers the 8 corners and writes its 3 partials to shared memory as [level][axis][point]
+// (conflict-free), then one thread per point sums its levels in order and stores dL/dx.
+// ---------------------------------------------------------------------------------------
+__host__ __device__ constexpr size_t input_grad_smem_bytes(int BP, int L, int F) {
+    return tile_smem_bytes(BP, L, F) + sizeof(float) * (size_t)BP * L * 3;
+}
+
+template <int F, typename TT, int BP>
+__global__ void __launch_bounds__(512, 2) backward_input_kernel(LevelParams lp, const float* __restrict__ x,
+                                                                const float* __restrict__ dout, int64_t N,
+                                                                const TT* __restrict__ table,
+                                                                float* __restrict__ dx) {
+    extern __shared__ __align__(16) float smem[];
+    const int L = lp.L;
+    const int W = L * F;
+    const int S = W + row_pad(F);
+    float* xs = smem;
+    float* gs = smem + BP * 3;
+    float* part = gs + BP * S;  // [L][3][BP]
+    const int64_t p0 = (int64_t)blockIdx.x * BP;
+    const int nvalid = (int)min((int64_t)BP, N - p0);
+
+    for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = __ldcs(x + p0 * 3 + i);
+    stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const int items = (BP / 32) * L;
+    for (int it = warp; it < items; it += nwarps) {
+        const int q = it / L;
+        const int l = it - q * L;
+        const int pl = q * 32 + lane;
+        if (pl < nvalid) {
+            Corners cr;
+            locate_corners(xs[pl * 3 + 0], xs[pl * 3 + 1], xs[pl * 3 + 2], lp.scale[l], lp.mask, cr);
+            const TT* tl = table + (uint64_t)l * lp.T * F;
+            float e[8][F];
+            gather_corners<F, TT, kGatherCorner>(tl, cr, e);
+            float g[F];
+            load_smem_entry<F>(gs + pl * S + l * F, g);
+            float sc[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float t = g[0] * e[c][0];
+#pragma unroll
+                for (int f = 1; f < F; ++f) t = fmaf(g[f], e[c][f], t);
+                sc[c] = t;
+            }
+            const float w0[2] = {1.0f - cr.f[0], cr.f[0]};
+            const float w1[2] = {1.0f - cr.f[1], cr.f[1]};
+            const float w2[2] = {1.0f - cr.f[2], cr.f[2]};
+            float d0 = 0.f, d1 = 0.f, d2 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const int b0 = c & 1, b1 = (c >> 1) & 1, b2 = (c >> 2) & 1;
+                const float s0 = b0 ? sc[c] : -sc[c];
+                const float s1 = b1 ? sc[c] : -sc[c];
+                const float s2 = b2 ? sc[c] : -sc[c];
+                d0 = fmaf(s0, w1[b1] * w2[b2], d0);
+                d1 = fmaf(s1, w0[b0] * w2[b2], d1);
+                d2 = fmaf(s2, w0[b0] * w1[b1], d2);
+            }
+            const float n = lp.scale[l];
+            part[(l * 3 + 0) * BP + pl] = n * d0;
+            part[(l * 3 + 1) * BP + pl] = n * d1;
+            part[(l * 3 + 2) * BP + pl] = n * d2;
+        }
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < nvalid * 3; t += blockDim.x) {
+        const int pt = t / 3, i = t - 3 * (t / 3);
+        float s = 0.f;
+        for (int l = 0; l < L; ++l) s += part[(l * 3 + i) * BP + pt];
+        __stcs(dx + p0 * 3 + t, s);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Sparse Adam on the tables ([NeRFace-HG] sections 3-4: Adam, no weight decay, only the
+// sampled entries receive gradient). Per element with nonzero gradient g:
+//   m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) g^2;
+//   theta -= lr * (m * c1) / (sqrt(v * c2) + eps),  c1 = 1/(1 - b1^t), c2 = 1/(1 - b2^t);
+// elements with g == 0 are left unchanged. Optionally the consumed gradient is zeroed,
+// which replaces a separate clear of the whole gradient table before the next backward.
+// Elementwise over L*T*F elements (a multiple of 16), 4 per thread, grid-stride; a group
+// of 4 zero gradients costs one 16-byte read.
+// ---------------------------------------------------------------------------------------
+struct AdamParams {
+    float lr, b1, b2, eps, c1, c2;
+};
+
+__device__ __forceinline__ float adam_one(float& m, float& v, float theta, float g, const AdamParams& a) {
+    m = fmaf(a.b1, m, (1.0f - a.b1) * g);
+    v = fmaf(a.b2, v, (1.0f - a.b2) * g * g);
+    const float denom = __fadd_rn(__fsqrt_rn(v * a.c2), a.eps);
+    return theta - a.lr * __fdiv_rn(m * a.c1, denom);
+}
+
+template <typename TT>
+__global__ void __launch_bounds__(256) adam_kernel(TT* __restrict__ param, float* __restrict__ mom1,
+                                                   float* __restrict__ mom2, float* __restrict__ grad,
+                                                   int64_t n4, AdamParams a, int zero_grad) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 g = __ldcs(reinterpret_cast<const float4*>(grad) + i);
+        if (g.x == 0.f && g.y == 0.f && g.z == 0.f && g.w == 0.f) continue;
+        float4 m = reinterpret_cast<float4*>(mom1)[i];
+        float4 v = reinterpret_cast<float4*>(mom2)[i];
+        float th[4];
+        if constexpr (sizeof(TT) == 4) {
+            const float4 t = reinterpret_cast<const float4*>(param)[i];
+            th[0] = t.x; th[1] = t.y; th[2] = t.z; th[3] = t.w;
+        } else {
+            const uint2 t = reinterpret_cast<const uint2*>(param)[i];
+            const float2 lo = h2_bits_to_f2(t.x), hi = h2_bits_to_f2(t.y);
+            th[0] = lo.x; th[1] = lo.y; th[2] = hi.x; th[3] = hi.y;
+        }
+        const float gv[4] = {g.x, g.y, g.z, g.w};
+        float mv[4] = {m.x, m.y, m.z, m.w}, vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (gv[k] != 0.f) th[k] = adam_one(mv[k], vv[k], th[k], gv[k], a);
+        reinterpret_cast<float4*>(mom1)[i] = make_float4(mv[0], mv[1], mv[2], mv[3]);
+        reinterpret_cast<float4*>(mom2)[i] = make_float4(vv[0], vv[1], vv[2], vv[3]);
+        if constexpr (sizeof(TT) == 4) {
+            reinterpret_cast<float4*>(param)[i] = make_float4(th[0], th[1], th[2], th[3]);
+        } else {
+            const __half2 lo = __floats2half2_rn(th[0], th[1]), hi = __floats2half2_rn(th[2], th[3]);
+            uint2 t;
+            t.x = *reinterpret_cast<const uint32_t*>(&lo);
+            t.y = *reinterpret_cast<const uint32_t*>(&hi);
+            reinterpret_cast<uint2*>(param)[i] = t;
+        }
+        if (zero_grad) __stcs(reinterpret_cast<float4*>(grad) + i, make_float4(0.f, 0.f, 0.f, 0.f));
+    }
 }
 
 // ---------------------------------------------------------------------------------------

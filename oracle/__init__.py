@@ -41,6 +41,11 @@ def _lib():
         lib.oracle_forward.restype = None
         lib.oracle_backward.argtypes = [i32, i32, i32, vp, vp, vp, i64, i32, i32, vp, i32]
         lib.oracle_backward.restype = None
+        lib.oracle_backward_x.argtypes = [i32, i32, i32, vp, i32, vp, vp, vp, i64, i32, i32, vp, i32]
+        lib.oracle_backward_x.restype = None
+        dbl = ctypes.c_double
+        lib.oracle_adam_step.argtypes = [i64, vp, vp, vp, vp, i64, dbl, dbl, dbl, dbl]
+        lib.oracle_adam_step.restype = None
         _LIB = lib
     return _LIB
 
@@ -71,6 +76,19 @@ def hash3(c0: int, c1: int, c2: int) -> int:
 def half_to_double(bits: int) -> float:
     """IEEE binary16 bit pattern -> float, decoded from the format's definition."""
     return float(_lib().oracle_half_to_double(int(bits) & 0xFFFF))
+
+
+def adam_step(param: np.ndarray, m: np.ndarray, v: np.ndarray, grad: np.ndarray, step: int,
+              lr: float, beta1: float = 0.9, beta2: float = 0.99, eps: float = 1e-15):
+    """Sparse Adam (NeRFace-HG sections 3-4): fp64 copies of param/m/v updated where the
+    fp32 gradient is nonzero. Returns (param, m, v) as new fp64 arrays."""
+    p = np.array(param, dtype=np.float64).ravel()
+    mm = np.array(m, dtype=np.float64).ravel()
+    vv = np.array(v, dtype=np.float64).ravel()
+    g = np.ascontiguousarray(grad, dtype=np.float32).ravel()
+    assert p.size == mm.size == vv.size == g.size
+    _lib().oracle_adam_step(p.size, _ptr(p), _ptr(mm), _ptr(vv), _ptr(g), int(step), lr, beta1, beta2, eps)
+    return p, mm, vv
 
 
 class Grid:
@@ -129,3 +147,17 @@ class Grid:
         _lib().oracle_backward(self.L, self.F, self.log2T, _ptr(self.res), _ptr(x), _ptr(g), N,
                                l0, l1, _ptr(dtable), nthreads)
         return dtable
+
+    def backward_x(self, x: np.ndarray, table: np.ndarray, g: np.ndarray, levels=None,
+                   nthreads: int = 1) -> np.ndarray:
+        """fp64 [N, 3] gradient of <g, encoding> with respect to x (NeRFace-HG section 3;
+        derivative of the trilinear weights inside the voxel that contains x)."""
+        x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1, 3)
+        table = self._check_table(table)
+        g = np.ascontiguousarray(g, dtype=np.float32).reshape(x.shape[0], self.L * self.F)
+        N = x.shape[0]
+        l0, l1 = self._levels(levels)
+        dx = np.zeros((N, 3), dtype=np.float64)
+        _lib().oracle_backward_x(self.L, self.F, self.log2T, _ptr(self.res), self.dtype, _ptr(table),
+                                 _ptr(x), _ptr(g), N, l0, l1, _ptr(dx), nthreads)
+        return dx

@@ -240,3 +240,80 @@ void oracle_backward(int L, int F, int log2T, const int *res, const float *x, co
         }
     }
 }
+
+/* ------------------------------------------------------------------------------------ */
+/* Backward pass with respect to the input coordinates. [NeRFace-HG] section 3 applies    */
+/* the encoder to coordinates produced by a learned transform, which needs dL/dx. Inside */
+/* the voxel that floor() selects, frac_i = x_i * N_l - v_i, so d frac_i / d x_i = N_l,  */
+/* and the weight of corner c changes along axis i by                                    */
+/*   d w_c / d x_i = N_l * (d_i ? +1 : -1) * prod_{j != i} (d_j ? frac_j : 1 - frac_j).  */
+/* (On a voxel face the encoding is continuous but has a kink; this is the derivative    */
+/* from the voxel that contains x, i.e. the one-sided derivative towards +x.)             */
+/*   dL_dx[p][i] = sum_l sum_c sum_f dL_dout[p][l*F + f] * table[l][idx_c][f] * dw_c/dx_i */
+/* Overwrites dx [N][3] (fp64). Levels l0 <= l < l1 are summed.                           */
+/* ------------------------------------------------------------------------------------ */
+void oracle_backward_x(int L, int F, int log2T, const int *res, int dtype, const void *table,
+                       const float *x, const float *g, int64_t N, int l0, int l1, double *dx,
+                       int nthreads)
+{
+    size_t T = (size_t)1 << log2T;
+    uint32_t mask = (uint32_t)(T - 1);
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+    for (int64_t p = 0; p < N; ++p) {
+        double acc[3] = {0.0, 0.0, 0.0};
+        for (int l = l0; l < l1; ++l) {
+            int64_t v[3], vc[3];
+            double frac[3];
+            locate(x + 3 * p, res[l], v, frac);
+            for (int c = 0; c < 8; ++c) {
+                (void)corner(v, frac, c, vc);
+                uint32_t h = oracle_hash3(vc[0], vc[1], vc[2]) & mask;
+                double ge = 0.0;  /* sum_f g * e_c[f] */
+                for (int f = 0; f < F; ++f)
+                    ge += (double)g[(size_t)p * L * F + (size_t)l * F + f] *
+                          table_value(table, dtype, ((size_t)l * T + h) * F + f);
+                for (int i = 0; i < 3; ++i) {
+                    double dw = (double)res[l] * (((c >> i) & 1) ? 1.0 : -1.0);
+                    for (int j = 0; j < 3; ++j) {
+                        if (j == i)
+                            continue;
+                        dw *= ((c >> j) & 1) ? frac[j] : 1.0 - frac[j];
+                    }
+                    acc[i] += ge * dw;
+                }
+            }
+        }
+        for (int i = 0; i < 3; ++i)
+            dx[3 * p + i] = acc[i];
+    }
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Sparse Adam step on the tables. [NeRFace-HG] sections 3 and 4: the tables are trained  */
+/* with Adam, without weight decay, at a learning rate several times the MLP's; only the  */
+/* sampled entries receive gradient in a step. [Overview-HG] sections 4-5: Adam, learning */
+/* rate 1e-2 to 1e-3. Adam (Kingma and Ba), for step t >= 1:                               */
+/*   m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) g^2;                                     */
+/*   theta -= lr * (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps).                        */
+/* Reading taken for "sparse": an element whose gradient is exactly zero was not sampled */
+/* in this step and is left entirely unchanged (theta, m and v). All fp64.               */
+/* param/m/v are updated in place (fp64 arrays of n elements).                           */
+/* ------------------------------------------------------------------------------------ */
+void oracle_adam_step(int64_t n, double *param, double *m, double *v, const float *grad,
+                      int64_t step, double lr, double beta1, double beta2, double eps)
+{
+    double c1 = 1.0 - pow(beta1, (double)step);
+    double c2 = 1.0 - pow(beta2, (double)step);
+    for (int64_t i = 0; i < n; ++i) {
+        double g = (double)grad[i];
+        if (g == 0.0)
+            continue;
+        m[i] = beta1 * m[i] + (1.0 - beta1) * g;
+        v[i] = beta2 * v[i] + (1.0 - beta2) * g * g;
+        double mhat = m[i] / c1;
+        double vhat = v[i] / c2;
+        param[i] -= lr * mhat / (sqrt(vhat) + eps);
+    }
+}

@@ -155,6 +155,24 @@ def test_calls_validate_before_any_launch():
         hg.hashgrid_destroy(h)
 
 
+def test_adam_and_input_gradient_validate_arguments():
+    h = hg.hashgrid_create(4, 2, 10, 2, 16)
+    try:
+        L = hg.lib
+        f = ctypes.c_float
+        assert L.hashgrid_adam_step(h, 0x1000, 0x1000, 0x1000, 0x1000, 0, f(1e-2), f(0.9), f(0.99), f(1e-15), 1, None) == hg.HASHGRID_ERR_ARG
+        assert L.hashgrid_adam_step(h, 0x1000, 0x1000, 0x1000, 0x1000, 1, f(1e-2), f(1.0), f(0.99), f(1e-15), 1, None) == hg.HASHGRID_ERR_ARG
+        assert L.hashgrid_adam_step(h, 0x1000, 0x1000, 0x1000, 0x1000, 1, f(1e-2), f(0.9), f(0.99), f(0.0), 1, None) == hg.HASHGRID_ERR_ARG
+        assert L.hashgrid_adam_step(h, None, 0x1000, 0x1000, 0x1000, 1, f(1e-2), f(0.9), f(0.99), f(1e-15), 1, None) == hg.HASHGRID_ERR_ARG
+        assert L.hashgrid_adam_step(None, 0x1000, 0x1000, 0x1000, 0x1000, 1, f(1e-2), f(0.9), f(0.99), f(1e-15), 1, None) == hg.HASHGRID_ERR_ARG
+        assert L.hashgrid_backward_input(h, None, None, 0, None, None, None) == hg.HASHGRID_OK
+        assert L.hashgrid_backward_input(h, 0x1004, 0x1000, 3, 0x1000, 0x1000, None) == hg.HASHGRID_ERR_ALIGN
+        a = np.zeros(4096, dtype=np.float32)
+        assert L.hashgrid_backward_input(h, a.ctypes.data, a.ctypes.data, 3, a.ctypes.data, a.ctypes.data, None) == hg.HASHGRID_ERR_ARG
+    finally:
+        hg.hashgrid_destroy(h)
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     """A copy of the binding with no built library beside it must raise ImportError on
     import: there is no fallback path."""

@@ -26,6 +26,12 @@ MUTATIONS = {
     "scale_by_N_minus_1": ("float xs = xp[i] * (float)res_l;", "float xs = xp[i] * (float)(res_l - 1);"),
     "literal_double_floor": ("if (fabs(v - r) <= 1e-9 * v)", "if (0)"),
     "overwrite_not_add": ("dtable[((size_t)l * T + h) * F + f] +=", "dtable[((size_t)l * T + h) * F + f] ="),
+    "dx_weight_sign": ("double dw = (double)res[l] * (((c >> i) & 1) ? 1.0 : -1.0);",
+                       "double dw = (double)res[l] * (((c >> i) & 1) ? -1.0 : 1.0);"),
+    "dx_missing_resolution": ("double dw = (double)res[l] * (((c >> i) & 1) ? 1.0 : -1.0);",
+                              "double dw = 1.0 * (((c >> i) & 1) ? 1.0 : -1.0);"),
+    "adam_no_bias_correction": ("double mhat = m[i] / c1;", "double mhat = m[i];"),
+    "adam_not_sparse": ("        if (g == 0.0)\n            continue;\n        m[i]", "        m[i]"),
     "int64_hash_low_bits_lost": ("return (u0 * ORACLE_PRIME_X) ^ (u1 * ORACLE_PRIME_Y) ^ (u2 * ORACLE_PRIME_Z);",
                                  "return ((u0 * ORACLE_PRIME_X) ^ (u1 * ORACLE_PRIME_Y) ^ (u2 * ORACLE_PRIME_Z)) & 0x7fffffffu;"),
 }
@@ -52,7 +58,7 @@ def test_pins_catch_mutation(tmp_path, name, monkeypatch):
     good = oracle._lib()                      # typed prototypes of the real library
     mut = ctypes.CDLL(path)
     for fn in ("oracle_resolutions", "oracle_hash3", "oracle_half_to_double", "oracle_indices",
-               "oracle_forward", "oracle_backward"):
+               "oracle_forward", "oracle_backward", "oracle_backward_x", "oracle_adam_step"):
         getattr(mut, fn).argtypes = getattr(good, fn).argtypes
         getattr(mut, fn).restype = getattr(good, fn).restype
     monkeypatch.setattr(oracle, "_LIB", mut)

@@ -351,3 +351,122 @@ def test_indices_match_bigint_hash():
             for c in range(8):
                 cc = [v[i] + ((c >> i) & 1) for i in range(3)]
                 assert idx[p, l, c] == bigint_hash(*cc, T=grid.T)
+
+
+# ---------------------------------------------------------------------------------------
+# Gradient with respect to the coordinates
+# ---------------------------------------------------------------------------------------
+
+def test_backward_x_finite_differences_exact():
+    """Inside a voxel the encoding is linear along each axis (trilinear = multilinear), so
+    a central difference is the derivative up to rounding. On the 2->16 grid (powers of
+    two) with x = (k + 1/2)/32 and h = 2^-12, every x*N_l and (x +- h)*N_l is exact in fp32
+    and x +- h stays inside the same voxel at every level."""
+    g = Grid(4, 2, 10, 2, 16)
+    rng = np.random.default_rng(21)
+    table = rng.standard_normal((4, 1024, 2)).astype(np.float32)
+    k = rng.integers(0, 32, size=(40, 3))
+    x = ((k + 0.5) / 32.0).astype(np.float32)
+    up = rng.standard_normal((40, 8)).astype(np.float32)
+    dx = g.backward_x(x, table, up)
+    h = np.float32(2.0 ** -12)
+    for i in range(3):
+        xp, xm = x.copy(), x.copy()
+        xp[:, i] += h
+        xm[:, i] -= h
+        fd = np.sum(up.astype(np.float64) * (g.forward(xp, table) - g.forward(xm, table)), axis=1) / (2 * float(h))
+        np.testing.assert_allclose(dx[:, i], fd, rtol=1e-9, atol=1e-9)
+
+
+def test_backward_x_constant_table_is_zero():
+    """A constant table gives a constant encoding: the weight derivatives of the 8 corners
+    sum to zero along every axis."""
+    g = Grid(4, 4, 10, 2, 16)
+    rng = np.random.default_rng(22)
+    x = rng.random((300, 3), dtype=np.float32)
+    up = rng.standard_normal((300, 16)).astype(np.float32)
+    dx = g.backward_x(x, np.full((4, 1024, 4), 0.75, dtype=np.float32), up)
+    assert np.max(np.abs(dx)) <= 1e-12
+
+
+def test_backward_x_affine_table_reproduced():
+    """Trilinear interpolation reproduces affine functions: with table[l][h(v)] = A v
+    (integer A, no hash collision among the grid's vertices at T = 2^20) the encoding at
+    level l is A (x N_l), so dL/dx_i = sum_l sum_f g[l, f] A[f, i] N_l exactly."""
+    g = Grid(3, 2, 20, 2, 8)
+    rng = np.random.default_rng(23)
+    A = rng.integers(-3, 4, size=(2, 3)).astype(np.float64)
+    table = np.zeros((3, g.T, 2), dtype=np.float32)
+    for l, n in enumerate(g.res):
+        seen = set()
+        for v in np.ndindex(n + 2, n + 2, n + 2):
+            h = bigint_hash(*v, T=g.T)
+            assert h not in seen, "hash collision among grid vertices"
+            seen.add(h)
+            table[l, h] = (A @ np.array(v, dtype=np.float64)).astype(np.float32)
+    x = rng.random((200, 3), dtype=np.float32)
+    up = rng.standard_normal((200, 6)).astype(np.float32)
+    want = np.zeros((200, 3))
+    for l, n in enumerate(g.res):
+        want += float(n) * (up[:, 2 * l:2 * l + 2].astype(np.float64) @ A)
+    np.testing.assert_allclose(g.backward_x(x, table, up), want, rtol=1e-12, atol=1e-9)
+
+
+# ---------------------------------------------------------------------------------------
+# Sparse Adam
+# ---------------------------------------------------------------------------------------
+
+def test_adam_untouched_elements_unchanged():
+    """An element with zero gradient was not sampled: parameter, m and v stay as they are."""
+    rng = np.random.default_rng(30)
+    p, m, v = rng.standard_normal(100), rng.standard_normal(100), rng.random(100)
+    g = np.zeros(100, dtype=np.float32)
+    p2, m2, v2 = oracle.adam_step(p, m, v, g, step=7, lr=1e-2)
+    np.testing.assert_array_equal(p2, p)
+    np.testing.assert_array_equal(m2, m)
+    np.testing.assert_array_equal(v2, v)
+
+
+def test_adam_first_step_closed_form():
+    """From m = v = 0 at t = 1 the bias corrections give m_hat = g and v_hat = g^2, so the
+    step is lr * g / (|g| + eps)."""
+    rng = np.random.default_rng(31)
+    p = rng.standard_normal(1000)
+    g = rng.standard_normal(1000).astype(np.float32)
+    p2, m2, v2 = oracle.adam_step(p, np.zeros(1000), np.zeros(1000), g, step=1, lr=0.01, beta1=0.9,
+                                  beta2=0.99, eps=1e-8)
+    gd = g.astype(np.float64)
+    np.testing.assert_allclose(p2, p - 0.01 * gd / (np.abs(gd) + 1e-8), rtol=1e-14, atol=1e-16)
+    np.testing.assert_allclose(m2, 0.1 * gd, rtol=1e-15)
+    np.testing.assert_allclose(v2, 0.01 * gd * gd, rtol=1e-13)
+
+
+def test_adam_constant_gradient_closed_form():
+    """With a constant gradient the bias-corrected moments stay exactly g and g^2, so after
+    t steps theta = theta_0 - t * lr * g / (|g| + eps)."""
+    rng = np.random.default_rng(32)
+    p0 = rng.standard_normal(200)
+    g = rng.standard_normal(200).astype(np.float32)
+    p, m, v = p0.copy(), np.zeros(200), np.zeros(200)
+    for t in range(1, 6):
+        p, m, v = oracle.adam_step(p, m, v, g, step=t, lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-12)
+    gd = g.astype(np.float64)
+    np.testing.assert_allclose(p, p0 - 5 * 1e-3 * gd / (np.abs(gd) + 1e-12), rtol=1e-12, atol=1e-14)
+
+
+def test_adam_matches_torch_adam_where_touched():
+    """Where every gradient is nonzero the sparse step is torch.optim.Adam without weight
+    decay (a library implementation of the same textbook update), in fp64."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(33)
+    p0 = rng.standard_normal(500)
+    prm = torch.nn.Parameter(torch.tensor(p0, dtype=torch.float64))
+    opt = torch.optim.Adam([prm], lr=5e-3, betas=(0.9, 0.99), eps=1e-10, weight_decay=0.0)
+    p, m, v = p0.copy(), np.zeros(500), np.zeros(500)
+    for t in range(1, 4):
+        g = (rng.standard_normal(500).astype(np.float32) + 0.25).astype(np.float32)
+        g[g == 0] = 1.0
+        prm.grad = torch.tensor(g.astype(np.float64))
+        opt.step()
+        p, m, v = oracle.adam_step(p, m, v, g, step=t, lr=5e-3, beta1=0.9, beta2=0.99, eps=1e-10)
+    np.testing.assert_allclose(p, prm.detach().numpy(), rtol=1e-12, atol=1e-14)

@@ -341,3 +341,134 @@ print("ok")
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
+
+
+# ---------------------------------------------------------------------------------------
+# Gradient with respect to the coordinates
+# ---------------------------------------------------------------------------------------
+
+def check_backward_x(og, x, table, g, got):
+    """|gpu - ref| <= 1e-5 * B_i, B_i = sum_l N_l * 2 * sum_f |g[l, f]| * max|table|: a bound
+    on the sum of absolute values of the terms (the 8 corner weight derivatives along one
+    axis have absolute sum 2 * N_l). fp32 products and sums stay within ~30 ulp of it."""
+    ref = og.backward_x(x, table, g, nthreads=THREADS)
+    tmax = float(np.max(np.abs(np.asarray(table, dtype=np.float64))))
+    F = og.F
+    B = np.zeros(x.shape[0])
+    for l, n in enumerate(og.res):
+        B += float(n) * 2.0 * np.sum(np.abs(g[:, l * F:(l + 1) * F].astype(np.float64)), axis=1) * tmax
+    err = np.abs(got.astype(np.float64) - ref)
+    lim = 1e-5 * B[:, None] + 1e-30
+    bad = np.argwhere(err > lim)
+    assert bad.size == 0, f"{len(bad)} off; first {bad[:3].tolist()}"
+
+
+@pytest.mark.parametrize("name", list(workloads.WORKLOADS))
+def test_backward_input_parity(name, reduced_inputs):
+    w, inp = reduced_inputs(name)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype)
+    got = grid.backward_input(dev(inp.x), dev(inp.g), dev(inp.table))
+    torch.cuda.synchronize()
+    check_backward_x(og, inp.x, inp.table, inp.g, got.cpu().numpy())
+
+
+@pytest.mark.parametrize("F", [1, 2, 4, 8])
+@pytest.mark.parametrize("dtype", ["f32", "f16"])
+def test_backward_input_widths_edges(F, dtype):
+    grid, og = make_pair(5, F, 12, 3, 200, dtype)
+    rng = np.random.default_rng(40 + F)
+    table = workloads.table_values(rng, 5, 2**12, F, dtype)
+    vals = np.array([0.0, 1.0 - 2**-24, 1.0, 0.5, -0.3, 1.7], dtype=np.float32)
+    xe = np.stack(np.meshgrid(vals, vals, vals, indexing="ij"), -1).reshape(-1, 3)
+    x = np.concatenate([workloads.uniform_points(rng, 777), xe]).astype(np.float32)
+    g = workloads.upstream_grads(rng, x.shape[0], 5 * F)
+    got = grid.backward_input(dev(x), dev(g), dev(table))
+    torch.cuda.synchronize()
+    check_backward_x(og, x, table, g, got.cpu().numpy())
+
+
+def test_backward_input_full_size_sampled():
+    """2^20 ray samples through the library's launch configuration; sampled rows checked."""
+    w = workloads.WORKLOADS["rays_L16F2T19"]
+    inp = workloads.make_inputs(w, seed=0)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max)
+    got = grid.backward_input(dev(inp.x), dev(inp.g), dev(inp.table)).cpu().numpy()
+    rows = np.unique(np.concatenate([np.random.default_rng(3).choice(inp.x.shape[0], 3000, replace=False),
+                                     np.arange(70), np.arange(inp.x.shape[0] - 70, inp.x.shape[0])]))
+    check_backward_x(og, inp.x[rows], inp.table, inp.g[rows], got[rows])
+
+
+# ---------------------------------------------------------------------------------------
+# Sparse Adam
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f32", "f16"])
+@pytest.mark.parametrize("zero_grad", [True, False])
+def test_adam_step_parity(dtype, zero_grad):
+    """Three steps on a sparse gradient (70% exact zeros). Each step starts the oracle from
+    the GPU's current state, so the check is per step: m and v within 1e-6 of
+    (|old| + |input term|), the parameter within 1e-6 * (|theta| + |step|) for fp32
+    (a few fp32 roundings in the update) or one fp16 ulp for fp16 tables; untouched
+    elements bit-identical; the gradient zeroed exactly when asked."""
+    hg = hgmod()
+    L, F, log2T = 4, 2, 12
+    grid, _ = make_pair(L, F, log2T, 2, 64, dtype)
+    rng = np.random.default_rng(50)
+    table = workloads.table_values(rng, L, 2**log2T, F, dtype)
+    n = table.size
+    t_d = dev(table)
+    m_d = torch.zeros(n, device="cuda")
+    v_d = torch.zeros(n, device="cuda")
+    lr, b1, b2, eps = 1e-2, 0.9, 0.99, 1e-15
+    for step in range(1, 4):
+        g = rng.standard_normal(n).astype(np.float32)
+        g[rng.random(n) < 0.7] = 0.0
+        g_d = dev(g)
+        p_in = t_d.cpu().numpy().astype(np.float64).ravel()
+        m_in, v_in = m_d.cpu().numpy().astype(np.float64), v_d.cpu().numpy().astype(np.float64)
+        hg.hashgrid_adam_step(grid.handle, t_d, m_d, v_d, g_d, step, lr, b1, b2, eps, zero_grad)
+        torch.cuda.synchronize()
+        p_ref, m_ref, v_ref = oracle.adam_step(p_in, m_in, v_in, g, step, lr, b1, b2, eps)
+        p_got = t_d.cpu().numpy().astype(np.float64).ravel()
+        m_got, v_got = m_d.cpu().numpy().astype(np.float64), v_d.cpu().numpy().astype(np.float64)
+        touched = g != 0
+        np.testing.assert_array_equal(p_got[~touched], p_in[~touched])
+        np.testing.assert_array_equal(m_got[~touched], m_in[~touched])
+        np.testing.assert_array_equal(v_got[~touched], v_in[~touched])
+        gd = g.astype(np.float64)
+        assert np.all(np.abs(m_got - m_ref) <= 1e-6 * (np.abs(m_in) + np.abs(gd)) + 1e-30)
+        assert np.all(np.abs(v_got - v_ref) <= 1e-6 * (np.abs(v_in) + gd * gd) + 1e-30)
+        if dtype == "f32":
+            lim = 1e-6 * (np.abs(p_ref) + np.abs(p_ref - p_in)) + 1e-30
+        else:
+            spacing = np.maximum(np.abs(p_ref), 2.0**-14) * 2.0**-10   # one fp16 ulp (subnormals: 2^-24)
+            lim = spacing + 1e-6 * np.abs(p_ref - p_in)
+        assert np.all(np.abs(p_got - p_ref) <= lim), float(np.max(np.abs(p_got - p_ref) - lim))
+        g_after = g_d.cpu().numpy()
+        if zero_grad:
+            assert np.all(g_after == 0)
+        else:
+            np.testing.assert_array_equal(g_after, g)
+
+
+def test_training_step_with_fused_clear():
+    """forward -> backward -> Adam (with the fused gradient clear), twice, on the ray
+    workload's grid: the second backward accumulates into the gradient the first Adam step
+    cleared, and matches the oracle's fresh gradient."""
+    hg = hgmod()
+    w = workloads.WORKLOADS["rays_L16F2T19"]
+    inp = workloads.make_inputs(w, seed=9, n_points=5000)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max)
+    x_d, t_d, g_d = dev(inp.x), dev(inp.table), dev(inp.g)
+    n = inp.table.size
+    m_d, v_d = torch.zeros(n, device="cuda"), torch.zeros(n, device="cuda")
+    dt = torch.zeros((w.L, w.T, w.F), device="cuda")
+    for step in (1, 2):
+        grid.forward(x_d, t_d)
+        grid.backward(x_d, g_d, dt)
+        torch.cuda.synchronize()
+        ref = og.backward(inp.x, inp.g, nthreads=THREADS)
+        assert rel_l2(dt.cpu().numpy(), ref) <= BWD_REL_L2
+        hg.hashgrid_adam_step(grid.handle, t_d, m_d, v_d, dt, step, 1e-2)
+        torch.cuda.synchronize()
+        assert float(dt.abs().max()) == 0.0
