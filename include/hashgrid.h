@@ -181,6 +181,30 @@ int hashgrid_adam_step(hashgrid_t h, void *table, float *adam_m, float *adam_v, 
                        void *cuda_stream);
 
 /*
+ * hashgrid_mlp_forward -- the encoding fused with the small MLP that consumes it, on the
+ * tensor cores.
+ *
+ * [NeRFace-HG] section 3: a three-layer network of 64 units with ReLU follows the hash
+ * features; [Repro-HG] section 4: Linear(in, 64), ReLU, Linear(64, 64), ReLU,
+ * Linear(64, 4). With e = the encoding of x (as hashgrid_forward computes it, L*F values):
+ *   y = W3 relu(W2 relu(W1 e + b1) + b2) + b3.
+ * The encoding stays on chip; each layer runs on the tcgen05 tensor cores over tiles of
+ * 128 points with bf16 operands (the encoding and the hidden activations are rounded to
+ * bf16) and fp32 accumulation. The pages' extra MLP inputs (an expression code, raw x)
+ * are not part of this call.
+ *
+ * x: [N,3] fp32; table: [L,T,F] of the handle's dtype; w1: [64][L*F], w2: [64][64],
+ * w3: [4][64] bf16 (uint16 bit patterns), row-major [out][in] like a torch Linear weight;
+ * b1: [64], b2: [64], b3: [4] fp32; y: [N,4] fp32 (overwritten). L*F must be 16, 32, 48
+ * or 64 (HASHGRID_ERR_ARG otherwise). device_status: NULL or a device int the caller sets
+ * to 0; the kernel sets it to 1 if it gave up waiting for the tensor cores (it then stops
+ * early and y is incomplete).
+ */
+int hashgrid_mlp_forward(hashgrid_t h, const float *x, int64_t N, const void *table, const void *w1,
+                         const float *b1, const void *w2, const float *b2, const void *w3,
+                         const float *b3, float *y, int *device_status, void *cuda_stream);
+
+/*
  * hashgrid_debug_indices -- export the hash index of every corner: idx_out[(p*L + l)*8 + c]
  * = index_c of point p at level l (uint32, < T), computed by the same device code as the
  * forward and backward passes. For tests and inspection. idx_out: [N, L, 8] uint32.

@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "hashgrid_backward_input": (i32, [vp, vp, vp, i64, vp, vp, vp]),
         "hashgrid_adam_step": (i32, [vp, vp, vp, vp, vp, i64, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                      ctypes.c_float, i32, vp]),
+        "hashgrid_mlp_forward": (i32, [vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "hashgrid_debug_indices": (i32, [vp, vp, i64, vp, vp]),
         "hashgrid_last_error": (ctypes.c_char_p, []),
         "hashgrid_version": (ctypes.c_char_p, []),
@@ -170,6 +171,12 @@ def hashgrid_adam_step(h: int, table, adam_m, adam_v, dL_dtable, step: int, lr: 
                        beta2: float = 0.99, eps: float = 1e-15, zero_grad: bool = True, stream=None) -> None:
     _check(lib.hashgrid_adam_step(h, _ptr(table), _ptr(adam_m), _ptr(adam_v), _ptr(dL_dtable), step, lr, beta1,
                                   beta2, eps, 1 if zero_grad else 0, _stream(stream)))
+
+
+def hashgrid_mlp_forward(h: int, x, N: int, table, w1, b1, w2, b2, w3, b3, y, device_status=None,
+                         stream=None) -> None:
+    _check(lib.hashgrid_mlp_forward(h, _ptr(x), N, _ptr(table), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(w3),
+                                    _ptr(b3), _ptr(y), _ptr(device_status), _stream(stream)))
 
 
 def hashgrid_debug_indices(h: int, x, N: int, idx_out, stream=None) -> None:

@@ -18,6 +18,7 @@
 
 #include "hashgrid.h"
 #include "hg_device.cuh"
+#include "hg_mlp.cuh"
 
 #define HASHGRID_VERSION_STRING "hashgrid-b200 0.1 (sm_100a)"
 
@@ -270,6 +271,42 @@ int launch_backward_input(const hashgrid_s* h, const float* x, const float* dout
     return launch_status("backward_input");
 }
 
+template <int F, typename TT, int K1>
+int launch_mlp_forward(const hashgrid_s* h, const float* x, int64_t N, const void* table, const void* w1,
+                       const float* b1, const void* w2, const float* b2, const void* w3, const float* b3, float* y,
+                       int* status, cudaStream_t s) {
+    auto k = hg::mlp::mlp_forward_kernel<F, TT, K1>;
+    const size_t smem = hg::mlp::smem_bytes(K1);
+    if (int rc = prepare_smem(k, smem)) return rc;
+    int dev = 0, sms = 148, per_sm = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, hg::mlp::kThreads, smem) != cudaSuccess || per_sm < 1) {
+        cudaGetLastError();
+        per_sm = 1;
+    }
+    const int64_t tiles = (N + hg::mlp::kM - 1) / hg::mlp::kM;
+    const int64_t cap = (int64_t)sms * per_sm;
+    const unsigned blocks = (unsigned)(tiles < cap ? tiles : cap);
+    k<<<blocks, hg::mlp::kThreads, smem, s>>>(h->lp, x, N, static_cast<const TT*>(table),
+                                               static_cast<const uint16_t*>(w1), b1, static_cast<const uint16_t*>(w2),
+                                               b2, static_cast<const uint16_t*>(w3), b3, y, status);
+    return launch_status("mlp_forward");
+}
+
+template <int F, typename TT>
+int dispatch_mlp_forward(const hashgrid_s* h, const float* x, int64_t N, const void* table, const void* w1,
+                         const float* b1, const void* w2, const float* b2, const void* w3, const float* b3, float* y,
+                         int* status, cudaStream_t s) {
+    switch (h->L * F) {
+        case 16: return launch_mlp_forward<F, TT, 16>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, status, s);
+        case 32: return launch_mlp_forward<F, TT, 32>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, status, s);
+        case 48: return launch_mlp_forward<F, TT, 48>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, status, s);
+        case 64: return launch_mlp_forward<F, TT, 64>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, status, s);
+    }
+    return fail(HASHGRID_ERR_ARG, "the MLP needs L*F in {16, 32, 48, 64}, got %d", h->L * F);
+}
+
 size_t table_bytes(const hashgrid_s* h) {
     return (size_t)h->L * ((size_t)1 << h->log2T) * (size_t)h->F * (h->dtype == HASHGRID_F16 ? 2 : 4);
 }
@@ -481,6 +518,42 @@ int hashgrid_adam_step(hashgrid_t h, void* table, float* adam_m, float* adam_v, 
     else
         hg::adam_kernel<float><<<blocks, 256, 0, s>>>(static_cast<float*>(table), adam_m, adam_v, dL_dtable, n4, a, zero_grad);
     return launch_status("adam_step");
+}
+
+int hashgrid_mlp_forward(hashgrid_t h, const float* x, int64_t N, const void* table, const void* w1,
+                         const float* b1, const void* w2, const float* b2, const void* w3, const float* b3, float* y,
+                         int* device_status, void* cuda_stream) {
+    if (int rc = check_handle(h)) return rc;
+    const int K1 = h->L * h->F;
+    if (K1 % 16 != 0 || K1 > 64)
+        return fail(HASHGRID_ERR_ARG, "the MLP needs L*F in {16, 32, 48, 64}, got %d", K1);
+    if (int rc = check_N(N, hg::mlp::kM)) return rc;
+    if (N == 0) return ok();
+    using namespace hg::mlp;
+    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(table, table_bytes(h), "table")) return rc;
+    if (int rc = check_buffer(w1, (size_t)kHid * K1 * 2, "w1")) return rc;
+    if (int rc = check_buffer(b1, kHid * sizeof(float), "b1")) return rc;
+    if (int rc = check_buffer(w2, (size_t)kHid * kHid * 2, "w2")) return rc;
+    if (int rc = check_buffer(b2, kHid * sizeof(float), "b2")) return rc;
+    if (int rc = check_buffer(w3, (size_t)kOut * kHid * 2, "w3")) return rc;
+    if (int rc = check_buffer(b3, kOut * sizeof(float), "b3")) return rc;
+    if (int rc = check_buffer(y, (size_t)N * kOut * sizeof(float), "y")) return rc;
+    if (device_status != nullptr)
+        if (int rc = check_buffer(device_status, sizeof(int), "device_status")) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    const bool half = h->dtype == HASHGRID_F16;
+    switch (h->F) {
+        case 1: return half ? dispatch_mlp_forward<1, __half>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, device_status, s)
+                            : dispatch_mlp_forward<1, float>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, device_status, s);
+        case 2: return half ? dispatch_mlp_forward<2, __half>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, device_status, s)
+                            : dispatch_mlp_forward<2, float>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, device_status, s);
+        case 4: return half ? dispatch_mlp_forward<4, __half>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, device_status, s)
+                            : dispatch_mlp_forward<4, float>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, device_status, s);
+        case 8: return half ? dispatch_mlp_forward<8, __half>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, device_status, s)
+                            : dispatch_mlp_forward<8, float>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, device_status, s);
+    }
+    return fail(HASHGRID_ERR_ARG, "corrupt handle");
 }
 
 int hashgrid_debug_indices(hashgrid_t h, const float* x, int64_t N, uint32_t* idx_out, void* cuda_stream) {

@@ -46,6 +46,10 @@ def _lib():
         dbl = ctypes.c_double
         lib.oracle_adam_step.argtypes = [i64, vp, vp, vp, vp, i64, dbl, dbl, dbl, dbl]
         lib.oracle_adam_step.restype = None
+        lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_double.restype = ctypes.c_double
+        lib.oracle_mlp_forward.argtypes = [i32, i32, i32, vp, i32, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, i32]
+        lib.oracle_mlp_forward.restype = None
         _LIB = lib
     return _LIB
 
@@ -76,6 +80,11 @@ def hash3(c0: int, c1: int, c2: int) -> int:
 def half_to_double(bits: int) -> float:
     """IEEE binary16 bit pattern -> float, decoded from the format's definition."""
     return float(_lib().oracle_half_to_double(int(bits) & 0xFFFF))
+
+
+def bf16_to_double(bits: int) -> float:
+    """bfloat16 bit pattern -> float (the upper half of a binary32)."""
+    return float(_lib().oracle_bf16_to_double(int(bits) & 0xFFFF))
 
 
 def adam_step(param: np.ndarray, m: np.ndarray, v: np.ndarray, grad: np.ndarray, step: int,
@@ -161,3 +170,22 @@ class Grid:
         _lib().oracle_backward_x(self.L, self.F, self.log2T, _ptr(self.res), self.dtype, _ptr(table),
                                  _ptr(x), _ptr(g), N, l0, l1, _ptr(dx), nthreads)
         return dx
+
+    def mlp_forward(self, x: np.ndarray, table: np.ndarray, w1: np.ndarray, b1: np.ndarray, w2: np.ndarray,
+                    b2: np.ndarray, w3: np.ndarray, b3: np.ndarray, nthreads: int = 1) -> np.ndarray:
+        """fp64 [N, 4] = W3 relu(W2 relu(W1 enc(x) + b1) + b2) + b3 (NeRFace-HG section 3,
+        Repro-HG section 4). Weights: uint16 bf16 bit patterns [out][in]; biases fp32."""
+        x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1, 3)
+        table = self._check_table(table)
+        K = self.L * self.F
+        w1 = np.ascontiguousarray(w1, dtype=np.uint16).reshape(64, K)
+        w2 = np.ascontiguousarray(w2, dtype=np.uint16).reshape(64, 64)
+        w3 = np.ascontiguousarray(w3, dtype=np.uint16).reshape(4, 64)
+        b1 = np.ascontiguousarray(b1, dtype=np.float32).reshape(64)
+        b2 = np.ascontiguousarray(b2, dtype=np.float32).reshape(64)
+        b3 = np.ascontiguousarray(b3, dtype=np.float32).reshape(4)
+        N = x.shape[0]
+        y = np.zeros((N, 4), dtype=np.float64)
+        _lib().oracle_mlp_forward(self.L, self.F, self.log2T, _ptr(self.res), self.dtype, _ptr(table), _ptr(x), N,
+                                  _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2), _ptr(w3), _ptr(b3), _ptr(y), nthreads)
+        return y

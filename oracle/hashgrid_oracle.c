@@ -317,3 +317,62 @@ void oracle_adam_step(int64_t n, double *param, double *m, double *v, const floa
         param[i] -= lr * mhat / (sqrt(vhat) + eps);
     }
 }
+
+/* ------------------------------------------------------------------------------------ */
+/* bfloat16 -> double: the bf16 format is the upper 16 bits of an IEEE binary32 value.  */
+/* ------------------------------------------------------------------------------------ */
+double oracle_bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Encoding followed by the small MLP that consumes it. [NeRFace-HG] section 3: a three- */
+/* layer network of 64 units with ReLU after the hash features; [Repro-HG] section 4:     */
+/* Linear(in, 64), ReLU, Linear(64, 64), ReLU, Linear(64, 4). Here in = L*F (the encoding */
+/* alone; the pages' extra inputs -- expression code, raw x -- are the caller's):         */
+/*   a1 = relu(W1 e + b1), a2 = relu(W2 a1 + b2), y = W3 a2 + b3                         */
+/* Weights are bf16 bit patterns, row-major [out][in] (W1 [64][in], W2 [64][64],         */
+/* W3 [4][64]), biases fp32; everything is evaluated in fp64 on the fp64 encoding.       */
+/* y: [N][4] fp64.                                                                       */
+/* ------------------------------------------------------------------------------------ */
+void oracle_mlp_forward(int L, int F, int log2T, const int *res, int dtype, const void *table,
+                        const float *x, int64_t N, const uint16_t *w1, const float *b1,
+                        const uint16_t *w2, const float *b2, const uint16_t *w3, const float *b3,
+                        double *y, int nthreads)
+{
+    const int in = L * F, hid = 64, nout = 4;
+    double *e = (double *)malloc(sizeof(double) * (size_t)N * in);
+    if (e == NULL)
+        return;
+    oracle_forward(L, F, log2T, res, dtype, table, x, N, 0, L, e, nthreads);
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+    for (int64_t p = 0; p < N; ++p) {
+        double a1[64], a2[64];
+        const double *ep = e + (size_t)p * in;
+        for (int o = 0; o < hid; ++o) {
+            double s = (double)b1[o];
+            for (int k = 0; k < in; ++k)
+                s += oracle_bf16_to_double(w1[o * in + k]) * ep[k];
+            a1[o] = s > 0.0 ? s : 0.0;
+        }
+        for (int o = 0; o < hid; ++o) {
+            double s = (double)b2[o];
+            for (int k = 0; k < hid; ++k)
+                s += oracle_bf16_to_double(w2[o * hid + k]) * a1[k];
+            a2[o] = s > 0.0 ? s : 0.0;
+        }
+        for (int o = 0; o < nout; ++o) {
+            double s = (double)b3[o];
+            for (int k = 0; k < hid; ++k)
+                s += oracle_bf16_to_double(w3[o * hid + k]) * a2[k];
+            y[(size_t)p * nout + o] = s;
+        }
+    }
+    free(e);
+}

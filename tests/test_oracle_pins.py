@@ -470,3 +470,46 @@ def test_adam_matches_torch_adam_where_touched():
         opt.step()
         p, m, v = oracle.adam_step(p, m, v, g, step=t, lr=5e-3, beta1=0.9, beta2=0.99, eps=1e-10)
     np.testing.assert_allclose(p, prm.detach().numpy(), rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------------------
+# Encoding + MLP
+# ---------------------------------------------------------------------------------------
+
+def bf16_bits(a):
+    """Round-to-nearest-even fp32 -> bf16 bit patterns (numpy)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u >> 16) & 1) + 0x7FFF
+    return ((u + r) >> 16).astype(np.uint16)
+
+
+def bf16_values(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def test_bf16_decode():
+    bits = np.arange(0, 65536, 97, dtype=np.uint32).astype(np.uint16)
+    for b in bits:
+        want = bf16_values(np.array([b]))[0]
+        got = oracle.bf16_to_double(int(b))
+        assert (got == want) or (np.isnan(got) and np.isnan(want))
+
+
+def test_mlp_matches_numpy_matmuls():
+    """The MLP of the oracle is three numpy matmuls with ReLU on the oracle's own fp64
+    encoding and the exactly decoded bf16 weights (a library routine for each layer)."""
+    g = Grid(16, 2, 12, 16, 512)
+    rng = np.random.default_rng(60)
+    table = (rng.standard_normal((16, 2**12, 2)) * 0.5).astype(np.float32)
+    x = rng.random((300, 3), dtype=np.float32)
+    w1 = bf16_bits(rng.standard_normal((64, 32)) * 0.3)
+    w2 = bf16_bits(rng.standard_normal((64, 64)) * 0.2)
+    w3 = bf16_bits(rng.standard_normal((4, 64)) * 0.2)
+    b1, b2, b3 = (rng.standard_normal(n).astype(np.float32) * 0.1 for n in (64, 64, 4))
+    y = g.mlp_forward(x, table, w1, b1, w2, b2, w3, b3)
+    e = g.forward(x, table)
+    a1 = np.maximum(e @ bf16_values(w1).T + b1.astype(np.float64), 0.0)
+    a2 = np.maximum(a1 @ bf16_values(w2).T + b2.astype(np.float64), 0.0)
+    want = a2 @ bf16_values(w3).T + b3.astype(np.float64)
+    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
+    assert np.any(a1 == 0) and np.any(a1 > 0)           # ReLU active on both sides

@@ -472,3 +472,82 @@ def test_training_step_with_fused_clear():
         hg.hashgrid_adam_step(grid.handle, t_d, m_d, v_d, dt, step, 1e-2)
         torch.cuda.synchronize()
         assert float(dt.abs().max()) == 0.0
+
+
+# ---------------------------------------------------------------------------------------
+# Encoding + MLP on the tensor cores
+# ---------------------------------------------------------------------------------------
+
+def bf16_bits(a):
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + ((u >> 16) & 1) + 0x7FFF) >> 16).astype(np.uint16)
+
+
+def bf16_values(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def mlp_weights(rng, K):
+    w1 = bf16_bits(rng.standard_normal((64, K)) * (2.0 / K) ** 0.5)
+    w2 = bf16_bits(rng.standard_normal((64, 64)) * (2.0 / 64) ** 0.5)
+    w3 = bf16_bits(rng.standard_normal((4, 64)) * (1.0 / 64) ** 0.5)
+    b1, b2, b3 = (rng.standard_normal(n).astype(np.float32) * 0.1 for n in (64, 64, 4))
+    return w1, b1, w2, b2, w3, b3
+
+
+def check_mlp(og, x, table, wts, got):
+    """|gpu - ref| <= 2 Ey + 1e-6. With u = 2^-8 (twice the bf16 rounding bound) the error
+    of each bf16 operand is propagated through |W|: E0 = u|e|,
+    E1 = |W1|E0 + u(|W1||e| + |b1|), E2 = |W2|E1 + u(|W2||a1| + |b2|),
+    Ey = |W3|E2 + 1e-6(|W3||a2| + |b3|) (fp32 accumulation), on the exact activations."""
+    w1, b1, w2, b2, w3, b3 = wts
+    ref = og.mlp_forward(x, table, *wts, nthreads=THREADS)
+    e = og.forward(x, table, nthreads=THREADS)
+    W1, W2, W3 = (np.abs(bf16_values(w)) for w in (w1, w2, w3))
+    a1 = np.maximum(e @ bf16_values(w1).T + b1, 0)
+    a2 = np.maximum(a1 @ bf16_values(w2).T + b2, 0)
+    u = 2.0 ** -8
+    E1 = np.abs(e) @ W1.T * u + u * (np.abs(e) @ W1.T + np.abs(b1))
+    E2 = E1 @ W2.T + u * (a1 @ W2.T + np.abs(b2))
+    Ey = E2 @ W3.T + 1e-6 * (a2 @ W3.T + np.abs(b3))
+    err = np.abs(got.astype(np.float64) - ref)
+    lim = 2 * Ey + 1e-6
+    bad = np.argwhere(err > lim)
+    assert bad.size == 0, f"{len(bad)} of {err.size} off; first {bad[:3].tolist()} err {err[tuple(bad[0])]:.3e} lim {lim[tuple(bad[0])]:.3e} ref {ref[tuple(bad[0])]:.3e} got {got[tuple(bad[0])]:.3e}"
+
+
+@pytest.mark.parametrize("shape", [(16, 2, 19, 16, 512, "f32"), (8, 2, 12, 4, 128, "f32"), (24, 2, 12, 4, 600, "f32"),
+                                   (16, 4, 14, 16, 4096, "f32"), (16, 2, 19, 16, 512, "f16")])
+def test_mlp_forward_parity(shape):
+    hg = hgmod()
+    L, F, log2T, a, b, dtype = shape
+    grid, og = make_pair(L, F, log2T, a, b, dtype)
+    rng = np.random.default_rng(70 + L * F)
+    table = (rng.standard_normal((L, 2**log2T, F)) * 0.3).astype(np.float32)
+    if dtype == "f16":
+        table = table.astype(np.float16)
+    x = np.concatenate([workloads.ray_points(rng, 40), workloads.uniform_points(rng, 1000)]).astype(np.float32)
+    wts = mlp_weights(rng, L * F)
+    N = x.shape[0]
+    y = torch.full((N, 4), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hg.hashgrid_mlp_forward(grid.handle, dev(x), N, dev(table), *[dev(w) for w in wts], y, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    check_mlp(og, x, table, wts, y.cpu().numpy())
+
+
+def test_mlp_forward_full_size_sampled():
+    hg = hgmod()
+    w = workloads.WORKLOADS["rays_L16F2T19"]
+    inp = workloads.make_inputs(w, seed=0, grads=False)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max)
+    rng = np.random.default_rng(71)
+    table = (inp.table * 3000).astype(np.float32)       # features of order 0.3, as after training
+    wts = mlp_weights(rng, 32)
+    N = inp.x.shape[0]
+    y = torch.empty((N, 4), device="cuda")
+    hg.hashgrid_mlp_forward(grid.handle, dev(inp.x), N, dev(table), *[dev(w) for w in wts], y)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([rng.choice(N, 3000, replace=False), np.arange(130), np.arange(N - 130, N)]))
+    check_mlp(og, inp.x[rows], table, wts, y.cpu().numpy()[rows])
