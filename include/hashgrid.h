@@ -140,6 +140,24 @@ int hashgrid_backward(hashgrid_t h, const float *x, const float *dL_dout, int64_
                       float *dL_dtable, void *cuda_stream);
 
 /*
+ * hashgrid_backward_half -- hashgrid_backward into an fp16 gradient table.
+ *
+ * The same contributions as hashgrid_backward (computed in fp32, merged in fp32 registers
+ * by the run walk), rounded to fp16 and reduced with packed 16-byte
+ * red.global.add.noftz.v4.f16x2 (round to nearest, subnormals kept): half the gradient
+ * memory, and two x-corners share one reduction more often (for F = 2, 3 x-pairs in 4).
+ * Each reduction rounds the running sum to fp16, so the result is accurate to about
+ * 2^-11 * sqrt(contributions per entry) relative; values beyond fp16 range overflow to
+ * infinity. Backward modes: ATOMIC = per-point reductions, every other mode = run
+ * merging; the schedule option applies.
+ *
+ * x: [N,3] fp32; dL_dout: [N,L*F] fp32; dL_dtable: [L,T,F] fp16 (IEEE binary16),
+ * ACCUMULATED into.
+ */
+int hashgrid_backward_half(hashgrid_t h, const float *x, const float *dL_dout, int64_t N,
+                           void *dL_dtable, void *cuda_stream);
+
+/*
  * hashgrid_backward_input -- gradient of a loss with respect to the input coordinates.
  *
  * [NeRFace-HG] section 3 applies the encoder to coordinates produced by a learned

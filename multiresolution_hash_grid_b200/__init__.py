@@ -69,6 +69,7 @@ def _load() -> ctypes.CDLL:
         "hashgrid_forward": (i32, [vp, vp, i64, vp, vp, vp]),
         "hashgrid_backward": (i32, [vp, vp, vp, i64, vp, vp]),
         "hashgrid_backward_input": (i32, [vp, vp, vp, i64, vp, vp, vp]),
+        "hashgrid_backward_half": (i32, [vp, vp, vp, i64, vp, vp]),
         "hashgrid_adam_step": (i32, [vp, vp, vp, vp, vp, i64, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                      ctypes.c_float, i32, vp]),
         "hashgrid_mlp_forward": (i32, [vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
@@ -161,6 +162,10 @@ def hashgrid_forward(h: int, x, N: int, table, out, stream=None) -> None:
 
 def hashgrid_backward(h: int, x, dL_dout, N: int, dL_dtable, stream=None) -> None:
     _check(lib.hashgrid_backward(h, _ptr(x), _ptr(dL_dout), N, _ptr(dL_dtable), _stream(stream)))
+
+
+def hashgrid_backward_half(h: int, x, dL_dout, N: int, dL_dtable, stream=None) -> None:
+    _check(lib.hashgrid_backward_half(h, _ptr(x), _ptr(dL_dout), N, _ptr(dL_dtable), _stream(stream)))
 
 
 def hashgrid_backward_input(h: int, x, dL_dout, N: int, table, dL_dx, stream=None) -> None:

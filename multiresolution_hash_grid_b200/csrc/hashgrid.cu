@@ -178,16 +178,16 @@ int launch_forward(const hashgrid_s* h, const float* x, int64_t N, const void* t
     return launch_status("forward");
 }
 
-template <int F, int kMode>
+template <int F, int kMode, typename GT = float>
 int launch_backward_mode(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
-                         float* dtable, cudaStream_t s) {
+                         GT* dtable, cudaStream_t s) {
     const int cap = hg::backward_threads(kMode);
     const int threads = tile_threads(h->L) < cap ? tile_threads(h->L) : cap;
     const size_t smem = hg::tile_smem_bytes(kTile, h->L, F) +
                         (kMode == hg::kAtomicOnly ? 0 : hg::group_smem_bytes(threads / 32, F));
     const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
     if constexpr (kMode == hg::kAtomicOnly) {
-        auto k = hg::backward_kernel_atomic<F, kTile>;
+        auto k = hg::backward_kernel_atomic<F, kTile, GT>;
         if (int rc = prepare_smem(k, smem)) return rc;
         k<<<blocks, threads, smem, s>>>(h->lp, x, dout, N, dtable);
     } else {
@@ -216,26 +216,27 @@ int launch_forward_levels(const hashgrid_s* h, const float* x, int64_t N, const 
     return launch_status("forward");
 }
 
-template <int F>
-int launch_backward_levels(const hashgrid_s* h, const float* x, const float* dout, int64_t N, float* dtable,
+// Run merging for every mode but ATOMIC (the warp-dedup modes have no level-major form).
+template <int F, typename GT>
+int launch_backward_levels(const hashgrid_s* h, const float* x, const float* dout, int64_t N, GT* dtable,
                            cudaStream_t s) {
     if constexpr (F <= 4) {
-        if (h->backward_mode == HASHGRID_BACKWARD_RUN_MERGE || h->backward_mode == HASHGRID_BACKWARD_AUTO) {
+        if (h->backward_mode != HASHGRID_BACKWARD_ATOMIC) {
             const int64_t runs = (N + hg::kRun - 1) / hg::kRun;
             const dim3 grid((unsigned)((runs + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
-            hg::backward_kernel_runs_levels<F><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, dout, N, dtable);
+            hg::backward_kernel_runs_levels<F, GT><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, dout, N, dtable);
             return launch_status("backward");
         }
     }
     const dim3 grid((unsigned)((N + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
-    hg::backward_kernel_atomic_levels<F><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, dout, N, dtable);
+    hg::backward_kernel_atomic_levels<F, GT><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, dout, N, dtable);
     return launch_status("backward");
 }
 
-template <int F>
+template <int F, typename GT = float>
 int launch_backward_runs(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
-                         float* dtable, cudaStream_t s) {
-    auto k = hg::backward_kernel_runs<F>;
+                         GT* dtable, cudaStream_t s) {
+    auto k = hg::backward_kernel_runs<F, GT>;
     const size_t smem = hg::run_smem_bytes(h->L, F);
     if (int rc = prepare_smem(k, smem)) return rc;
     const unsigned blocks = (unsigned)((N + hg::kRunTile - 1) / hg::kRunTile);
@@ -243,12 +244,23 @@ int launch_backward_runs(const hashgrid_s* h, const float* x, const float* dout,
     return launch_status("backward");
 }
 
+// fp16 gradient tables: run merging (every mode but ATOMIC) or per-point reductions.
+template <int F>
+int launch_backward_half(const hashgrid_s* h, const float* x, const float* dout, int64_t N, __half* dtable,
+                         cudaStream_t s) {
+    if (level_major(h)) return launch_backward_levels<F, __half>(h, x, dout, N, dtable, s);
+    if constexpr (F <= 4) {
+        if (h->backward_mode != HASHGRID_BACKWARD_ATOMIC) return launch_backward_runs<F, __half>(h, x, dout, N, dtable, s);
+    }
+    return launch_backward_mode<F, hg::kAtomicOnly, __half>(h, x, dout, N, dtable, s);
+}
+
 template <int F>
 int launch_backward(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
                     float* dtable, cudaStream_t s) {
     const bool grouped = h->backward_mode == HASHGRID_BACKWARD_WARP_DEDUP ||
                          h->backward_mode == HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE;
-    if (!grouped && level_major(h)) return launch_backward_levels<F>(h, x, dout, N, dtable, s);
+    if (!grouped && level_major(h)) return launch_backward_levels<F, float>(h, x, dout, N, dtable, s);
     if constexpr (F <= 4) {
         if (h->backward_mode == HASHGRID_BACKWARD_RUN_MERGE || h->backward_mode == HASHGRID_BACKWARD_AUTO)
             return launch_backward_runs<F>(h, x, dout, N, dtable, s);
@@ -278,13 +290,12 @@ int launch_mlp_forward(const hashgrid_s* h, const float* x, int64_t N, const voi
     auto k = hg::mlp::mlp_forward_kernel<F, TT, K1>;
     const size_t smem = hg::mlp::smem_bytes(K1);
     if (int rc = prepare_smem(k, smem)) return rc;
-    int dev = 0, sms = 148, per_sm = 1;
+    int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, hg::mlp::kThreads, smem) != cudaSuccess || per_sm < 1) {
-        cudaGetLastError();
-        per_sm = 1;
-    }
+    // Persistent grid: as many CTAs as fit per SM (registers and shared memory allow 3 for
+    // F <= 4, 2 for F = 8; TMEM holds 3 x 64 columns of 512). More would only queue.
+    const int per_sm = F == 8 ? 2 : 3;
     const int64_t tiles = (N + hg::mlp::kM - 1) / hg::mlp::kM;
     const int64_t cap = (int64_t)sms * per_sm;
     const unsigned blocks = (unsigned)(tiles < cap ? tiles : cap);
@@ -461,6 +472,26 @@ int hashgrid_backward(hashgrid_t h, const float* x, const float* dL_dout, int64_
         case 2: return launch_backward<2>(h, x, dL_dout, N, dL_dtable, s);
         case 4: return launch_backward<4>(h, x, dL_dout, N, dL_dtable, s);
         case 8: return launch_backward<8>(h, x, dL_dout, N, dL_dtable, s);
+    }
+    return fail(HASHGRID_ERR_ARG, "corrupt handle");
+}
+
+int hashgrid_backward_half(hashgrid_t h, const float* x, const float* dL_dout, int64_t N, void* dL_dtable,
+                           void* cuda_stream) {
+    if (int rc = check_handle(h)) return rc;
+    if (int rc = check_N(N, kTile)) return rc;
+    if (N == 0) return ok();
+    const size_t W = (size_t)h->L * h->F;
+    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(dL_dout, (size_t)N * W * sizeof(float), "dL_dout")) return rc;
+    if (int rc = check_buffer(dL_dtable, hashgrid_table_elems(h) * 2, "dL_dtable")) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    __half* d = static_cast<__half*>(dL_dtable);
+    switch (h->F) {
+        case 1: return launch_backward_half<1>(h, x, dL_dout, N, d, s);
+        case 2: return launch_backward_half<2>(h, x, dL_dout, N, d, s);
+        case 4: return launch_backward_half<4>(h, x, dL_dout, N, d, s);
+        case 8: return launch_backward_half<8>(h, x, dL_dout, N, d, s);
     }
     return fail(HASHGRID_ERR_ARG, "corrupt handle");
 }

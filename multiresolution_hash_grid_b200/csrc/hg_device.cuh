@@ -228,6 +228,50 @@ __device__ __forceinline__ void red_pair(float* dl, uint32_t a, uint32_t b, cons
     }
 }
 
+// fp16 gradient tables: 16-byte red.global.add.noftz.v4.f16x2 (sm_90+) on aligned units of
+// 8 halves (8 / F entries). Contributions are rounded to fp16 (round to nearest, subnormals
+// kept) and the L2 adds in fp16. Two x-corners share a unit more often than in fp32
+// (F = 2: when v0 mod 4 != 3), so fewer reductions reach L2.
+__device__ __forceinline__ void red_half_unit(__half* p, const float (&u)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        __half2 h = __floats2half2_rn(u[2 * k], u[2 * k + 1]);
+        w[k] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    asm volatile("red.global.add.noftz.v4.f16x2 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                 "r"(w[3])
+                 : "memory");
+}
+
+template <int F>
+__device__ __forceinline__ void unit_vals_half(uint32_t i, const float* v, float (&u)[8]) {
+    constexpr uint32_t kUnit = 8 / F;
+    const uint32_t o = (i & (kUnit - 1)) * F;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        float t = 0.f;
+#pragma unroll
+        for (int f = 0; f < F; ++f) t = (o + f == (uint32_t)k) ? v[f] : t;
+        u[k] = t;
+    }
+}
+
+template <int F>
+__device__ __forceinline__ void red_pair(__half* dl, uint32_t a, uint32_t b, const float* va, const float* vb,
+                                         bool ra = true, bool rb = true) {
+    constexpr uint32_t kUnit = 8 / F;
+    const bool shared = ra && rb && (a ^ b) < kUnit;
+    float ua[8], ub[8], u1[8];
+    unit_vals_half<F>(a, va, ua);
+    unit_vals_half<F>(b, vb, ub);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) u1[k] = shared ? ua[k] + ub[k] : (ra ? ua[k] : ub[k]);
+    const uint32_t i1 = ra ? a : b;
+    if (ra || rb) red_half_unit(dl + (uint64_t)(i1 & ~(kUnit - 1)) * F, u1);
+    if (ra && rb && !shared) red_half_unit(dl + (uint64_t)(b & ~(kUnit - 1)) * F, ub);
+}
+
 // ---------------------------------------------------------------------------------------
 // Voxel, corner indices and trilinear weights of one point at one level.
 // [NeRFace-HG] section 2: xs = x * N_l (one fp32 multiply, never fused), v = floor(xs),
@@ -616,10 +660,10 @@ struct GroupWarp {
 // warp): 3 blocks per SM, 2 for F = 4. The plain mode runs 16 warps per block.
 __host__ __device__ constexpr int backward_threads(int mode) { return mode == kAtomicOnly ? 512 : 256; }
 
-template <int F, int BP, int kMode>
+template <int F, int BP, int kMode, typename GT = float>
 __device__ __forceinline__ void backward_body(const LevelParams& lp, const float* __restrict__ x,
                                               const float* __restrict__ dout, int64_t N,
-                                              float* __restrict__ dtable) {
+                                              GT* __restrict__ dtable) {
     static_assert(kMode == kAtomicOnly || F <= 4, "grouped units are 16 bytes");
     extern __shared__ __align__(16) float smem[];
     const int L = lp.L;
@@ -647,7 +691,7 @@ __device__ __forceinline__ void backward_body(const LevelParams& lp, const float
         const int pl = q * 32 + lane;
         const bool valid = pl < nvalid;
         const int pc = valid ? pl : 0;  // rows past the tail read row 0 and contribute nothing
-        float* dl = dtable + (uint64_t)l * lp.T * F;
+        GT* dl = dtable + (uint64_t)l * lp.T * F;
         Corners cr;
         locate_corners(xs[pc * 3 + 0], xs[pc * 3 + 1], xs[pc * 3 + 2], lp.scale[l], lp.mask, cr);
         float g[F];
@@ -662,20 +706,25 @@ __device__ __forceinline__ void backward_body(const LevelParams& lp, const float
                               abs(cr.v[2] - u2) <= 1;
             group = __popc(__ballot_sync(0xffffffffu, near)) >= 16;
         }
-        if (group) {
-            const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-            if (valid) {
-                float v[8][FG];
+        if constexpr (kMode != kAtomicOnly) {
+            static_assert(sizeof(GT) == 4, "grouped reductions accumulate fp32 gradients");
+            if (group) {
+                const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+                if (valid) {
+                    float v[8][FG];
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
+                    for (int c = 0; c < 8; ++c)
 #pragma unroll
-                    for (int f = 0; f < FG; ++f) v[c][f] = cr.w[c] * g[f < F ? f : 0];
-                grp.push8(dl, cr.idx, v, lane, vmask);
+                        for (int f = 0; f < FG; ++f) v[c][f] = cr.w[c] * g[f < F ? f : 0];
+                    grp.push8(dl, cr.idx, v, lane, vmask);
+                }
+                __syncwarp();
+                grp.flush(dl, lane);
+                __syncwarp();
+                continue;
             }
-            __syncwarp();
-            grp.flush(dl, lane);
-            __syncwarp();
-        } else if (valid) {
+        }
+        if (valid) {
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
                 float va[F], vb[F];
@@ -690,11 +739,11 @@ __device__ __forceinline__ void backward_body(const LevelParams& lp, const float
     }
 }
 
-template <int F, int BP>
+template <int F, int BP, typename GT>
 __global__ void __launch_bounds__(512) backward_kernel_atomic(LevelParams lp, const float* __restrict__ x,
                                                               const float* __restrict__ dout, int64_t N,
-                                                              float* __restrict__ dtable) {
-    backward_body<F, BP, kAtomicOnly>(lp, x, dout, N, dtable);
+                                                              GT* __restrict__ dtable) {
+    backward_body<F, BP, kAtomicOnly, GT>(lp, x, dout, N, dtable);
 }
 
 template <int F, int BP, int kMode>
@@ -725,8 +774,8 @@ __host__ __device__ constexpr size_t run_smem_bytes(int L, int F) {
     return sizeof(float) * ((size_t)32 * run_x_stride() + (size_t)32 * run_g_stride(L, F));
 }
 
-template <int F>
-__device__ __forceinline__ void run_flush(float* dl, const float (&acc)[8][F], const uint32_t (&cidx)[8],
+template <int F, typename GT>
+__device__ __forceinline__ void run_flush(GT* dl, const float (&acc)[8][F], const uint32_t (&cidx)[8],
                                           int ax, uint32_t leave_bit) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -740,8 +789,8 @@ __device__ __forceinline__ void run_flush(float* dl, const float (&acc)[8][F], c
 // Walk one run of `n` consecutive points at one level (scale, mask) and reduce into the
 // level table dl. xp(j, x3) loads point j's 3 coordinates; gl(j, g) its F upstream
 // gradients.
-template <int F, class XP, class GL>
-__device__ __forceinline__ void walk_run(float* dl, float scale, uint32_t mask, int n, XP xp, GL gl) {
+template <int F, typename GT, class XP, class GL>
+__device__ __forceinline__ void walk_run(GT* dl, float scale, uint32_t mask, int n, XP xp, GL gl) {
     float acc[8][F];
     uint32_t cidx[8];
     int cv0 = 0, cv1 = 0, cv2 = 0;
@@ -794,10 +843,10 @@ __device__ __forceinline__ void walk_run(float* dl, float scale, uint32_t mask, 
     if (n > 0) run_flush<F>(dl, acc, cidx, -1, 0u);
 }
 
-template <int F>
+template <int F, typename GT>
 __global__ void __launch_bounds__(256) backward_kernel_runs(LevelParams lp, const float* __restrict__ x,
                                                            const float* __restrict__ dout, int64_t N,
-                                                           float* __restrict__ dtable) {
+                                                           GT* __restrict__ dtable) {
     static_assert(F <= 4, "run merging keeps 8 x F sums in registers");
     extern __shared__ __align__(16) float smem[];
     const int L = lp.L;
@@ -838,7 +887,7 @@ __global__ void __launch_bounds__(256) backward_kernel_runs(LevelParams lp, cons
     const int nwarps = blockDim.x >> 5;
     const int jmax = min(kRun, nvalid - lane * kRun);  // points of this lane's run (may be <= 0)
     for (int l = warp; l < L; l += nwarps) {
-        float* dl = dtable + (uint64_t)l * lp.T * F;
+        GT* dl = dtable + (uint64_t)l * lp.T * F;
         walk_run<F>(dl, lp.scale[l], lp.mask, jmax,
                     [&](int j, float* x3) {
                         const float* q = xs + lane * XS + j * 3;
@@ -955,10 +1004,10 @@ __global__ void __launch_bounds__(kLevelBlock) forward_kernel_levels(LevelParams
     store_global_entry<F>(out + p * (int64_t)(lp.L * F) + l * F, o);
 }
 
-template <int F>
+template <int F, typename GT>
 __global__ void __launch_bounds__(kLevelBlock) backward_kernel_atomic_levels(LevelParams lp, const float* __restrict__ x,
                                                                             const float* __restrict__ dout, int64_t N,
-                                                                            float* __restrict__ dtable) {
+                                                                            GT* __restrict__ dtable) {
     const int l = blockIdx.y;
     const int64_t p = (int64_t)blockIdx.x * kLevelBlock + threadIdx.x;
     if (p >= N) return;
@@ -966,7 +1015,7 @@ __global__ void __launch_bounds__(kLevelBlock) backward_kernel_atomic_levels(Lev
     locate_corners(__ldcs(x + p * 3), __ldcs(x + p * 3 + 1), __ldcs(x + p * 3 + 2), lp.scale[l], lp.mask, cr);
     float g[F];
     load_global_entry<F>(dout + p * (int64_t)(lp.L * F) + l * F, g);
-    float* dl = dtable + (uint64_t)l * lp.T * F;
+    GT* dl = dtable + (uint64_t)l * lp.T * F;
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) {
         float va[F], vb[F];
@@ -980,16 +1029,16 @@ __global__ void __launch_bounds__(kLevelBlock) backward_kernel_atomic_levels(Lev
 }
 
 // One thread walks one run of kRun consecutive points at level blockIdx.y.
-template <int F>
+template <int F, typename GT>
 __global__ void __launch_bounds__(kLevelBlock) backward_kernel_runs_levels(LevelParams lp, const float* __restrict__ x,
                                                                           const float* __restrict__ dout, int64_t N,
-                                                                          float* __restrict__ dtable) {
+                                                                          GT* __restrict__ dtable) {
     const int l = blockIdx.y;
     const int64_t p0 = ((int64_t)blockIdx.x * kLevelBlock + threadIdx.x) * kRun;
     if (p0 >= N) return;
     const int n = (int)min((int64_t)kRun, N - p0);
     const int64_t W = lp.L * F;
-    float* dl = dtable + (uint64_t)l * lp.T * F;
+    GT* dl = dtable + (uint64_t)l * lp.T * F;
     walk_run<F>(dl, lp.scale[l], lp.mask, n,
                 [&](int j, float* x3) {
                     const float* q = x + (p0 + j) * 3;

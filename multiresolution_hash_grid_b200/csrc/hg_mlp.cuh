@@ -10,7 +10,8 @@
 // the encoding and the hidden activations rounded to bf16 as MMA operands and fp32
 // accumulation in tensor memory. The encoding never leaves the SM.
 //
-// Persistent CTAs of 512 threads: the weights are staged in shared memory once; per tile of
+// Persistent CTAs of 512 threads, up to 3 per SM (3 x 64 of the 512 TMEM columns) so one
+// CTA's encoding overlaps another's MMAs: the weights are staged in shared memory once; per tile of
 // 128 points the 16 warps encode (4 threads per point, each a quarter of the levels) into
 // the bf16 A operand, one thread issues the layer's MMAs and commits them to an mbarrier,
 // and after the (bounded) wait the 16 warps read the accumulator rows back with
@@ -140,7 +141,7 @@ __device__ __forceinline__ void hidden_epilogue(uint32_t tmem, const float* bias
 }
 
 template <int F, typename TT, int K1>
-__global__ void __launch_bounds__(kThreads, 1) mlp_forward_kernel(
+__global__ void __launch_bounds__(kThreads, F == 8 ? 2 : 3) mlp_forward_kernel(
     LevelParams lp, const float* __restrict__ x, int64_t N, const TT* __restrict__ table,
     const uint16_t* __restrict__ w1, const float* __restrict__ b1, const uint16_t* __restrict__ w2,
     const float* __restrict__ b2, const uint16_t* __restrict__ w3, const float* __restrict__ b3,
@@ -202,12 +203,21 @@ __global__ void __launch_bounds__(kThreads, 1) mlp_forward_kernel(
                 locate_corners(x0, x1, x2, lp.scale[l], lp.mask, cr);
                 float e[8][F];
                 gather_corners<F, TT, kGatherCorner>(table + (uint64_t)l * lp.T * F, cr, e);
+                float o[F];
 #pragma unroll
                 for (int f = 0; f < F; ++f) {
                     float acc = cr.w[0] * e[0][f];
 #pragma unroll
                     for (int c = 1; c < 8; ++c) acc = fmaf(cr.w[c], e[c][f], acc);
-                    *reinterpret_cast<__nv_bfloat16*>(A0 + canon(pt, l * F + f, K1)) = __float2bfloat16_rn(acc);
+                    o[f] = acc;
+                }
+                if constexpr (F == 1) {
+                    *reinterpret_cast<__nv_bfloat16*>(A0 + canon(pt, l, K1)) = __float2bfloat16_rn(o[0]);
+                } else {
+                    // F even: the pairs (l*F + 2j, + 1) are adjacent within one core-matrix row
+#pragma unroll
+                    for (int j = 0; j < F / 2; ++j)
+                        *reinterpret_cast<uint32_t*>(A0 + canon(pt, l * F + 2 * j, K1)) = pack_bf16(o[2 * j], o[2 * j + 1]);
                 }
             }
         }

@@ -551,3 +551,58 @@ def test_mlp_forward_full_size_sampled():
     torch.cuda.synchronize()
     rows = np.unique(np.concatenate([rng.choice(N, 3000, replace=False), np.arange(130), np.arange(N - 130, N)]))
     check_mlp(og, inp.x[rows], table, wts, y.cpu().numpy()[rows])
+
+
+# ---------------------------------------------------------------------------------------
+# fp16 gradient tables (packed f16x2 reductions)
+# ---------------------------------------------------------------------------------------
+
+def check_half_gradient(og, x, g, got):
+    """fp16 accumulation model. Each reduction rounds its operand and the running sum to
+    fp16 (unit roundoff 2^-11, subnormal spacing 2^-24). With A_e = sum of |contributions|
+    into element e (the oracle's gradient of |g|, weights being >= 0) and n_e the number of
+    contributions: |err_e| <= 2^-11 (n_e + 1) A_e + 2^-24 (n_e + 1) (worst case), and per
+    level the relative L2 error <= 3 * 2^-11 sqrt(mean n_e) + 2^-11 (rounding errors of a
+    running sum add like a random walk)."""
+    ref = og.backward(x, g, nthreads=THREADS)
+    A = og.backward(x, np.abs(g), nthreads=THREADS)
+    idx = og.indices(x)
+    got = got.astype(np.float64)
+    u = 2.0 ** -11
+    for l in range(og.L):
+        n = np.bincount(idx[:, l, :].ravel(), minlength=og.T).astype(np.float64)[:, None]
+        err = np.abs(got[l] - ref[l])
+        lim = u * (n + 1) * A[l] + 2.0 ** -24 * (n + 1)
+        assert np.all(err <= lim), (l, float(np.max(err - lim)))
+        touched = n[:, 0] > 0
+        den = np.linalg.norm(ref[l][touched])
+        if den > 0:
+            rel = np.linalg.norm((got[l] - ref[l])[touched]) / den
+            assert rel <= 3 * u * np.sqrt(np.mean(n[touched])) + u, (l, rel)
+
+
+@pytest.mark.parametrize("mode", ["auto", "atomic", "runs/level", "atomic/level"])
+@pytest.mark.parametrize("name", ["tiny_L4F2T10", "rays_L16F2T19", "half_L16F2T19"])
+def test_backward_half_parity(name, mode, reduced_inputs):
+    hg = hgmod()
+    w, inp = reduced_inputs(name)
+    bm, _, sched = mode.partition("/")
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, w.dtype, backward=bm if bm != "auto" else "auto",
+                         schedule=sched or "point")
+    d = torch.zeros((w.L, w.T, w.F), dtype=torch.float16, device="cuda")
+    hg.hashgrid_backward_half(grid.handle, dev(inp.x), dev(inp.g), inp.x.shape[0], d)
+    torch.cuda.synchronize()
+    check_half_gradient(og, inp.x, inp.g, d.cpu().numpy())
+
+
+@pytest.mark.parametrize("F", [1, 4, 8])
+def test_backward_half_widths(F):
+    hg = hgmod()
+    grid, og = make_pair(5, F, 12, 3, 200)
+    rng = np.random.default_rng(80 + F)
+    x = workloads.uniform_points(rng, 2000)
+    g = workloads.upstream_grads(rng, 2000, 5 * F)
+    d = torch.zeros((5, 2**12, F), dtype=torch.float16, device="cuda")
+    hg.hashgrid_backward_half(grid.handle, dev(x), dev(g), 2000, d)
+    torch.cuda.synchronize()
+    check_half_gradient(og, x, g, d.cpu().numpy())
