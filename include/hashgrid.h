@@ -93,6 +93,25 @@ enum hashgrid_status {
  */
 int hashgrid_create(int L, int F, int log2T, int N_min, int N_max, int dtype, hashgrid_t *out);
 
+/*
+ * hashgrid_create_nd -- hashgrid_create for D-dimensional points, D in {2, 3, 4}.
+ *
+ * [Repro-HG] section 2.2 writes the hash for any dimension d as the XOR over axes of
+ * coordinate_i * pi_i (mod T) and section 3 lists the primes (1, 2654435761, 805459861,
+ * 3674653429, 2097192037, 1434869437, 2165219737); axis i uses the i-th. A point
+ * interpolates the 2^D corners of its cell with multilinear weights
+ * prod_i (offset_i ? frac_i : 1 - frac_i), corner c having offset bit i = (c >> i) & 1.
+ * x is then [N, D] and dL_dx [N, D]; hashgrid_debug_indices writes [N, L, 2^D].
+ * D = 3 is hashgrid_create. For D != 3 the forward pass gathers per corner and the backward
+ * passes reduce per point (the gather, backward-mode and schedule options apply to D = 3
+ * only), and hashgrid_mlp_forward is not available.
+ */
+int hashgrid_create_nd(int D, int L, int F, int log2T, int N_min, int N_max, int dtype,
+                       hashgrid_t *out);
+
+/* Input dimensions D of a handle (0 for a NULL handle). */
+int hashgrid_dims(hashgrid_t h);
+
 /* Free a handle (NULL is allowed). The caller must not destroy a handle while calls that
  * use it are still being issued from other threads; work already launched is unaffected. */
 int hashgrid_destroy(hashgrid_t h);

@@ -59,6 +59,8 @@ def _load() -> ctypes.CDLL:
     i32, i64, vp, sz = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
     protos = {
         "hashgrid_create": (i32, [i32, i32, i32, i32, i32, i32, ctypes.POINTER(vp)]),
+        "hashgrid_create_nd": (i32, [i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(vp)]),
+        "hashgrid_dims": (i32, [vp]),
         "hashgrid_destroy": (i32, [vp]),
         "hashgrid_resolutions": (i32, [vp, ctypes.POINTER(i32)]),
         "hashgrid_table_elems": (sz, [vp]),
@@ -120,6 +122,16 @@ def hashgrid_create(L: int, F: int, log2T: int, N_min: int, N_max: int, dtype: i
     h = ctypes.c_void_p()
     _check(lib.hashgrid_create(L, F, log2T, N_min, N_max, dtype, ctypes.byref(h)))
     return h.value
+
+
+def hashgrid_create_nd(D: int, L: int, F: int, log2T: int, N_min: int, N_max: int, dtype: int = HASHGRID_F32) -> int:
+    h = ctypes.c_void_p()
+    _check(lib.hashgrid_create_nd(D, L, F, log2T, N_min, N_max, dtype, ctypes.byref(h)))
+    return h.value
+
+
+def hashgrid_dims(h: int) -> int:
+    return int(lib.hashgrid_dims(h))
 
 
 def hashgrid_destroy(h: int) -> None:
@@ -195,10 +207,10 @@ class HashGrid:
 
     def __init__(self, L: int = 16, F: int = 2, log2T: int = 19, N_min: int = 16, N_max: int = 512,
                  dtype: int = HASHGRID_F32, forward_gather: int = HASHGRID_GATHER_AUTO,
-                 backward_mode: int = HASHGRID_BACKWARD_AUTO, schedule: int = HASHGRID_SCHEDULE_AUTO):
-        self.L, self.F, self.log2T, self.N_min, self.N_max, self.dtype = L, F, log2T, N_min, N_max, dtype
+                 backward_mode: int = HASHGRID_BACKWARD_AUTO, schedule: int = HASHGRID_SCHEDULE_AUTO, D: int = 3):
+        self.L, self.F, self.log2T, self.N_min, self.N_max, self.dtype, self.D = L, F, log2T, N_min, N_max, dtype, D
         self.T = 1 << log2T
-        self.handle = hashgrid_create(L, F, log2T, N_min, N_max, dtype)
+        self.handle = hashgrid_create_nd(D, L, F, log2T, N_min, N_max, dtype)
         hashgrid_set_option(self.handle, HASHGRID_OPT_FORWARD_GATHER, forward_gather)
         hashgrid_set_option(self.handle, HASHGRID_OPT_BACKWARD_MODE, backward_mode)
         hashgrid_set_option(self.handle, HASHGRID_OPT_SCHEDULE, schedule)
@@ -231,12 +243,12 @@ class HashGrid:
     def backward_input(self, x, dL_dout, table, dL_dx=None, stream=None):
         import torch
         if dL_dx is None:
-            dL_dx = torch.empty((x.shape[0], 3), dtype=torch.float32, device=x.device)
+            dL_dx = torch.empty((x.shape[0], self.D), dtype=torch.float32, device=x.device)
         hashgrid_backward_input(self.handle, x, dL_dout, x.shape[0], table, dL_dx, stream)
         return dL_dx
 
     def indices(self, x, stream=None):
         import torch
-        idx = torch.empty((x.shape[0], self.L, 8), dtype=torch.int32, device=x.device)
+        idx = torch.empty((x.shape[0], self.L, 1 << self.D), dtype=torch.int32, device=x.device)
         hashgrid_debug_indices(self.handle, x, x.shape[0], idx, stream)
         return idx

@@ -15,14 +15,17 @@
 #include <cstring>
 #include <new>
 #include <string>
+#include <type_traits>
 
 #include "hashgrid.h"
 #include "hg_device.cuh"
 #include "hg_mlp.cuh"
+#include "hg_nd.cuh"
 
 #define HASHGRID_VERSION_STRING "hashgrid-b200 0.1 (sm_100a)"
 
 struct hashgrid_s {
+    int D;  // input dimensions (3 for hashgrid_create)
     int L, F, log2T, N_min, N_max, dtype;
     int res[HASHGRID_MAX_LEVELS];
     int forward_gather;   // HASHGRID_GATHER_*
@@ -318,6 +321,48 @@ int dispatch_mlp_forward(const hashgrid_s* h, const float* x, int64_t N, const v
     return fail(HASHGRID_ERR_ARG, "the MLP needs L*F in {16, 32, 48, 64}, got %d", h->L * F);
 }
 
+// D-dimensional inputs (D = 2, 4): per-corner gathers and per-point reductions.
+template <int D, int F, typename TT>
+int launch_nd_forward(const hashgrid_s* h, const float* x, int64_t N, const void* table, float* out, cudaStream_t s) {
+    auto k = hg::nd::forward_kernel<D, F, TT>;
+    const size_t smem = hg::nd::tile_smem_bytes(D, h->L, F);
+    if (int rc = prepare_smem(k, smem)) return rc;
+    k<<<(unsigned)((N + hg::nd::kTile - 1) / hg::nd::kTile), tile_threads(h->L), smem, s>>>(
+        h->lp, x, N, static_cast<const TT*>(table), out);
+    return launch_status("forward");
+}
+
+template <int D, int F, typename GT>
+int launch_nd_backward(const hashgrid_s* h, const float* x, const float* dout, int64_t N, GT* dtable, cudaStream_t s) {
+    auto k = hg::nd::backward_kernel<D, F, GT>;
+    const size_t smem = hg::nd::tile_smem_bytes(D, h->L, F);
+    if (int rc = prepare_smem(k, smem)) return rc;
+    k<<<(unsigned)((N + hg::nd::kTile - 1) / hg::nd::kTile), tile_threads(h->L), smem, s>>>(h->lp, x, dout, N, dtable);
+    return launch_status("backward");
+}
+
+template <int D, int F, typename TT>
+int launch_nd_backward_input(const hashgrid_s* h, const float* x, const float* dout, int64_t N, const void* table,
+                             float* dx, cudaStream_t s) {
+    auto k = hg::nd::backward_input_kernel<D, F, TT>;
+    const size_t smem = hg::nd::tile_smem_bytes(D, h->L, F) + sizeof(float) * (size_t)hg::nd::kTile * h->L * D;
+    if (int rc = prepare_smem(k, smem)) return rc;
+    k<<<(unsigned)((N + hg::nd::kTile - 1) / hg::nd::kTile), tile_threads(h->L), smem, s>>>(
+        h->lp, x, dout, N, static_cast<const TT*>(table), dx);
+    return launch_status("backward_input");
+}
+
+// Calls fn<D, F>() for the handle's D (2 or 4) and F.
+template <class Fn>
+int nd_dispatch(const hashgrid_s* h, Fn&& fn) {
+#define HG_ND_CASE(DD, FF) \
+    if (h->D == DD && h->F == FF) return fn(std::integral_constant<int, DD>(), std::integral_constant<int, FF>());
+    HG_ND_CASE(2, 1) HG_ND_CASE(2, 2) HG_ND_CASE(2, 4) HG_ND_CASE(2, 8)
+    HG_ND_CASE(4, 1) HG_ND_CASE(4, 2) HG_ND_CASE(4, 4) HG_ND_CASE(4, 8)
+#undef HG_ND_CASE
+    return fail(HASHGRID_ERR_ARG, "corrupt handle");
+}
+
 size_t table_bytes(const hashgrid_s* h) {
     return (size_t)h->L * ((size_t)1 << h->log2T) * (size_t)h->F * (h->dtype == HASHGRID_F16 ? 2 : 4);
 }
@@ -346,6 +391,7 @@ int hashgrid_create(int L, int F, int log2T, int N_min, int N_max, int dtype, ha
     hashgrid_s* h = new (std::nothrow) hashgrid_s;
     if (h == nullptr) return fail(HASHGRID_ERR_OOM, "out of host memory");
     std::memset(h, 0, sizeof(*h));
+    h->D = 3;
     h->L = L; h->F = F; h->log2T = log2T; h->N_min = N_min; h->N_max = N_max; h->dtype = dtype;
     compute_resolutions(L, N_min, N_max, h->res);
     h->lp.L = L;
@@ -355,6 +401,16 @@ int hashgrid_create(int L, int F, int log2T, int N_min, int N_max, int dtype, ha
     *out = h;
     return ok();
 }
+
+int hashgrid_create_nd(int D, int L, int F, int log2T, int N_min, int N_max, int dtype, hashgrid_t* out) {
+    if (out != nullptr) *out = nullptr;
+    if (D != 2 && D != 3 && D != 4) return fail(HASHGRID_ERR_ARG, "D = %d is not 2, 3 or 4", D);
+    int rc = hashgrid_create(L, F, log2T, N_min, N_max, dtype, out);
+    if (rc == HASHGRID_OK) (*out)->D = D;
+    return rc;
+}
+
+int hashgrid_dims(hashgrid_t h) { return h == nullptr ? 0 : h->D; }
 
 int hashgrid_destroy(hashgrid_t h) {
     delete h;
@@ -428,11 +484,16 @@ int hashgrid_forward(hashgrid_t h, const float* x, int64_t N, const void* table,
     if (int rc = check_N(N, kTile)) return rc;
     if (N == 0) return ok();
     const size_t W = (size_t)h->L * h->F;
-    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(x, (size_t)N * h->D * sizeof(float), "x")) return rc;
     if (int rc = check_buffer(table, table_bytes(h), "table")) return rc;
     if (int rc = check_buffer(out, (size_t)N * W * sizeof(float), "out")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     const bool half = h->dtype == HASHGRID_F16;
+    if (h->D != 3)
+        return nd_dispatch(h, [&](auto d, auto f) {
+            return half ? launch_nd_forward<decltype(d)::value, decltype(f)::value, __half>(h, x, N, table, out, s)
+                        : launch_nd_forward<decltype(d)::value, decltype(f)::value, float>(h, x, N, table, out, s);
+        });
     // Sector gathers issue 256-bit loads, which need a 32-byte-aligned table.
     const bool aligned32 = reinterpret_cast<uintptr_t>(table) % 32 == 0;
     if (h->forward_gather == HASHGRID_GATHER_SECTOR && !aligned32)
@@ -463,10 +524,14 @@ int hashgrid_backward(hashgrid_t h, const float* x, const float* dL_dout, int64_
     if (int rc = check_N(N, kTile)) return rc;
     if (N == 0) return ok();
     const size_t W = (size_t)h->L * h->F;
-    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(x, (size_t)N * h->D * sizeof(float), "x")) return rc;
     if (int rc = check_buffer(dL_dout, (size_t)N * W * sizeof(float), "dL_dout")) return rc;
     if (int rc = check_buffer(dL_dtable, hashgrid_table_elems(h) * sizeof(float), "dL_dtable")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    if (h->D != 3)
+        return nd_dispatch(h, [&](auto d, auto f) {
+            return launch_nd_backward<decltype(d)::value, decltype(f)::value, float>(h, x, dL_dout, N, dL_dtable, s);
+        });
     switch (h->F) {
         case 1: return launch_backward<1>(h, x, dL_dout, N, dL_dtable, s);
         case 2: return launch_backward<2>(h, x, dL_dout, N, dL_dtable, s);
@@ -482,11 +547,15 @@ int hashgrid_backward_half(hashgrid_t h, const float* x, const float* dL_dout, i
     if (int rc = check_N(N, kTile)) return rc;
     if (N == 0) return ok();
     const size_t W = (size_t)h->L * h->F;
-    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(x, (size_t)N * h->D * sizeof(float), "x")) return rc;
     if (int rc = check_buffer(dL_dout, (size_t)N * W * sizeof(float), "dL_dout")) return rc;
     if (int rc = check_buffer(dL_dtable, hashgrid_table_elems(h) * 2, "dL_dtable")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     __half* d = static_cast<__half*>(dL_dtable);
+    if (h->D != 3)
+        return nd_dispatch(h, [&](auto dd, auto f) {
+            return launch_nd_backward<decltype(dd)::value, decltype(f)::value, __half>(h, x, dL_dout, N, d, s);
+        });
     switch (h->F) {
         case 1: return launch_backward_half<1>(h, x, dL_dout, N, d, s);
         case 2: return launch_backward_half<2>(h, x, dL_dout, N, d, s);
@@ -502,12 +571,18 @@ int hashgrid_backward_input(hashgrid_t h, const float* x, const float* dL_dout, 
     if (int rc = check_N(N, kTile)) return rc;
     if (N == 0) return ok();
     const size_t W = (size_t)h->L * h->F;
-    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(x, (size_t)N * h->D * sizeof(float), "x")) return rc;
     if (int rc = check_buffer(dL_dout, (size_t)N * W * sizeof(float), "dL_dout")) return rc;
     if (int rc = check_buffer(table, table_bytes(h), "table")) return rc;
-    if (int rc = check_buffer(dL_dx, (size_t)N * 3 * sizeof(float), "dL_dx")) return rc;
+    if (int rc = check_buffer(dL_dx, (size_t)N * h->D * sizeof(float), "dL_dx")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     const bool half = h->dtype == HASHGRID_F16;
+    if (h->D != 3)
+        return nd_dispatch(h, [&](auto d, auto f) {
+            constexpr int DD = decltype(d)::value, FF = decltype(f)::value;
+            return half ? launch_nd_backward_input<DD, FF, __half>(h, x, dL_dout, N, table, dL_dx, s)
+                        : launch_nd_backward_input<DD, FF, float>(h, x, dL_dout, N, table, dL_dx, s);
+        });
     switch (h->F) {
         case 1: return half ? launch_backward_input<1, __half>(h, x, dL_dout, N, table, dL_dx, s) : launch_backward_input<1, float>(h, x, dL_dout, N, table, dL_dx, s);
         case 2: return half ? launch_backward_input<2, __half>(h, x, dL_dout, N, table, dL_dx, s) : launch_backward_input<2, float>(h, x, dL_dout, N, table, dL_dx, s);
@@ -555,13 +630,14 @@ int hashgrid_mlp_forward(hashgrid_t h, const float* x, int64_t N, const void* ta
                          const float* b1, const void* w2, const float* b2, const void* w3, const float* b3, float* y,
                          int* device_status, void* cuda_stream) {
     if (int rc = check_handle(h)) return rc;
+    if (h->D != 3) return fail(HASHGRID_ERR_ARG, "the MLP takes 3-D points, the handle has D = %d", h->D);
     const int K1 = h->L * h->F;
     if (K1 % 16 != 0 || K1 > 64)
         return fail(HASHGRID_ERR_ARG, "the MLP needs L*F in {16, 32, 48, 64}, got %d", K1);
     if (int rc = check_N(N, hg::mlp::kM)) return rc;
     if (N == 0) return ok();
     using namespace hg::mlp;
-    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(x, (size_t)N * h->D * sizeof(float), "x")) return rc;
     if (int rc = check_buffer(table, table_bytes(h), "table")) return rc;
     if (int rc = check_buffer(w1, (size_t)kHid * K1 * 2, "w1")) return rc;
     if (int rc = check_buffer(b1, kHid * sizeof(float), "b1")) return rc;
@@ -591,14 +667,19 @@ int hashgrid_debug_indices(hashgrid_t h, const float* x, int64_t N, uint32_t* id
     if (int rc = check_handle(h)) return rc;
     if (int rc = check_N(N, 1)) return rc;
     if (N == 0) return ok();
-    if (int rc = check_buffer(x, (size_t)N * 3 * sizeof(float), "x")) return rc;
-    if (int rc = check_buffer(idx_out, (size_t)N * h->L * 8 * sizeof(uint32_t), "idx_out")) return rc;
+    if (int rc = check_buffer(x, (size_t)N * h->D * sizeof(float), "x")) return rc;
+    if (int rc = check_buffer(idx_out, (size_t)N * h->L * ((size_t)1 << h->D) * sizeof(uint32_t), "idx_out")) return rc;
     const int64_t total = N * h->L;
     const int threads = 256;
     const int64_t blocks = (total + threads - 1) / threads;
     if (blocks > 0x7fffffffLL) return fail(HASHGRID_ERR_ARG, "N too large for the index export");
-    hg::indices_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
-        h->lp, x, N, idx_out);
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    if (h->D == 2)
+        hg::nd::indices_kernel<2><<<(unsigned)blocks, threads, 0, s>>>(h->lp, x, N, idx_out);
+    else if (h->D == 4)
+        hg::nd::indices_kernel<4><<<(unsigned)blocks, threads, 0, s>>>(h->lp, x, N, idx_out);
+    else
+        hg::indices_kernel<<<(unsigned)blocks, threads, 0, s>>>(h->lp, x, N, idx_out);
     return launch_status("debug_indices");
 }
 

@@ -50,6 +50,16 @@ def _lib():
         lib.oracle_bf16_to_double.restype = ctypes.c_double
         lib.oracle_mlp_forward.argtypes = [i32, i32, i32, vp, i32, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, i32]
         lib.oracle_mlp_forward.restype = None
+        lib.oracle_hash_nd.argtypes = [i32, vp]
+        lib.oracle_hash_nd.restype = ctypes.c_uint32
+        lib.oracle_indices_nd.argtypes = [i32, i32, i32, vp, vp, i64, vp]
+        lib.oracle_indices_nd.restype = None
+        lib.oracle_forward_nd.argtypes = [i32, i32, i32, i32, vp, i32, vp, vp, i64, vp, i32]
+        lib.oracle_forward_nd.restype = None
+        lib.oracle_backward_nd.argtypes = [i32, i32, i32, i32, vp, vp, vp, i64, vp, i32]
+        lib.oracle_backward_nd.restype = None
+        lib.oracle_backward_x_nd.argtypes = [i32, i32, i32, i32, vp, i32, vp, vp, vp, i64, vp, i32]
+        lib.oracle_backward_x_nd.restype = None
         _LIB = lib
     return _LIB
 
@@ -80,6 +90,56 @@ def hash3(c0: int, c1: int, c2: int) -> int:
 def half_to_double(bits: int) -> float:
     """IEEE binary16 bit pattern -> float, decoded from the format's definition."""
     return float(_lib().oracle_half_to_double(int(bits) & 0xFFFF))
+
+
+def hash_nd(coords) -> int:
+    """uint32 hash of a D-dimensional vertex with the 7-prime list (Repro-HG sections 2.2, 3)."""
+    c = np.ascontiguousarray(np.asarray(coords, dtype=np.int64))
+    return int(_lib().oracle_hash_nd(c.size, _ptr(c)))
+
+
+class GridND:
+    """D-dimensional encoding (D in 2..7 for the hash; 2^D corners, multilinear weights)."""
+
+    def __init__(self, D: int, L: int, F: int, log2T: int, N_min: int, N_max: int, dtype: int = F32):
+        self.D, self.L, self.F, self.log2T, self.N_min, self.N_max, self.dtype = D, L, F, log2T, N_min, N_max, dtype
+        self.T = 1 << log2T
+        self.res = np.asarray(resolutions(L, N_min, N_max), dtype=np.int32)
+
+    def _x(self, x):
+        return np.ascontiguousarray(x, dtype=np.float32).reshape(-1, self.D)
+
+    def _table(self, table):
+        return Grid._check_table(self, table)
+
+    def indices(self, x):
+        x = self._x(x)
+        idx = np.zeros((x.shape[0], self.L, 1 << self.D), dtype=np.uint32)
+        _lib().oracle_indices_nd(self.D, self.L, self.log2T, _ptr(self.res), _ptr(x), x.shape[0], _ptr(idx))
+        return idx
+
+    def forward(self, x, table, nthreads: int = 1):
+        x, table = self._x(x), self._table(table)
+        out = np.zeros((x.shape[0], self.L * self.F))
+        _lib().oracle_forward_nd(self.D, self.L, self.F, self.log2T, _ptr(self.res), self.dtype, _ptr(table), _ptr(x),
+                                 x.shape[0], _ptr(out), nthreads)
+        return out
+
+    def backward(self, x, g, nthreads: int = 1):
+        x = self._x(x)
+        g = np.ascontiguousarray(g, dtype=np.float32).reshape(x.shape[0], self.L * self.F)
+        d = np.zeros((self.L, self.T, self.F))
+        _lib().oracle_backward_nd(self.D, self.L, self.F, self.log2T, _ptr(self.res), _ptr(x), _ptr(g), x.shape[0],
+                                  _ptr(d), nthreads)
+        return d
+
+    def backward_x(self, x, table, g, nthreads: int = 1):
+        x, table = self._x(x), self._table(table)
+        g = np.ascontiguousarray(g, dtype=np.float32).reshape(x.shape[0], self.L * self.F)
+        dx = np.zeros((x.shape[0], self.D))
+        _lib().oracle_backward_x_nd(self.D, self.L, self.F, self.log2T, _ptr(self.res), self.dtype, _ptr(table),
+                                    _ptr(x), _ptr(g), x.shape[0], _ptr(dx), nthreads)
+        return dx
 
 
 def bf16_to_double(bits: int) -> float:

@@ -376,3 +376,144 @@ void oracle_mlp_forward(int L, int F, int log2T, const int *res, int dtype, cons
     }
     free(e);
 }
+
+/* ------------------------------------------------------------------------------------ */
+/* D-dimensional inputs. [Repro-HG] section 2.2 writes the hash for coordinates of any   */
+/* dimension d as the XOR over axes of coordinate_i * pi_i, and section 3 lists the       */
+/* primes (1, 2654435761, 805459861, 3674653429, 2097192037, 1434869437, 2165219737);    */
+/* the encoding of a D-dimensional point interpolates the 2^D corners of its cell with   */
+/* multilinear weights prod_i (d_i ? frac_i : 1 - frac_i). Corner c has offset bit i =   */
+/* (c >> i) & 1. x is [N][D]. D = 3 reproduces the functions above.                       */
+/* ------------------------------------------------------------------------------------ */
+static const uint32_t ORACLE_PRIMES7[7] = {1u, 2654435761u, 805459861u, 3674653429u,
+                                           2097192037u, 1434869437u, 2165219737u};
+
+uint32_t oracle_hash_nd(int D, const int64_t *c)
+{
+    uint32_t h = 0;
+    for (int i = 0; i < D; ++i)
+        h ^= (uint32_t)c[i] * ORACLE_PRIMES7[i];
+    return h;
+}
+
+static void locate_nd(int D, const float *xp, int res_l, int64_t *v, double *frac)
+{
+    for (int i = 0; i < D; ++i) {
+        float xs = xp[i] * (float)res_l;
+        float fl = floorf(xs);
+        v[i] = (int64_t)fl;
+        frac[i] = (double)(xs - fl);
+    }
+}
+
+static double corner_nd(int D, const int64_t *v, const double *frac, int c, int64_t *vc)
+{
+    double w = 1.0;
+    for (int i = 0; i < D; ++i) {
+        int d = (c >> i) & 1;
+        vc[i] = v[i] + d;
+        w *= d ? frac[i] : 1.0 - frac[i];
+    }
+    return w;
+}
+
+void oracle_indices_nd(int D, int L, int log2T, const int *res, const float *x, int64_t N, uint32_t *idx)
+{
+    uint32_t mask = (uint32_t)((1ull << log2T) - 1ull);
+    int nc = 1 << D;
+    for (int64_t p = 0; p < N; ++p)
+        for (int l = 0; l < L; ++l) {
+            int64_t v[7], vc[7];
+            double frac[7];
+            locate_nd(D, x + (size_t)D * p, res[l], v, frac);
+            for (int c = 0; c < nc; ++c) {
+                (void)corner_nd(D, v, frac, c, vc);
+                idx[((size_t)p * L + l) * nc + c] = oracle_hash_nd(D, vc) & mask;
+            }
+        }
+}
+
+void oracle_forward_nd(int D, int L, int F, int log2T, const int *res, int dtype, const void *table,
+                       const float *x, int64_t N, double *out, int nthreads)
+{
+    size_t T = (size_t)1 << log2T;
+    uint32_t mask = (uint32_t)(T - 1);
+    int nc = 1 << D;
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+    for (int64_t p = 0; p < N; ++p)
+        for (int l = 0; l < L; ++l) {
+            int64_t v[7], vc[7];
+            double frac[7], acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            locate_nd(D, x + (size_t)D * p, res[l], v, frac);
+            for (int c = 0; c < nc; ++c) {
+                double w = corner_nd(D, v, frac, c, vc);
+                uint32_t h = oracle_hash_nd(D, vc) & mask;
+                for (int f = 0; f < F; ++f)
+                    acc[f] += w * table_value(table, dtype, ((size_t)l * T + h) * F + f);
+            }
+            for (int f = 0; f < F; ++f)
+                out[(size_t)p * L * F + (size_t)l * F + f] = acc[f];
+        }
+}
+
+void oracle_backward_nd(int D, int L, int F, int log2T, const int *res, const float *x, const float *g,
+                        int64_t N, double *dtable, int nthreads)
+{
+    size_t T = (size_t)1 << log2T;
+    uint32_t mask = (uint32_t)(T - 1);
+    int nc = 1 << D;
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int l = 0; l < L; ++l)
+        for (int64_t p = 0; p < N; ++p) {
+            int64_t v[7], vc[7];
+            double frac[7];
+            locate_nd(D, x + (size_t)D * p, res[l], v, frac);
+            for (int c = 0; c < nc; ++c) {
+                double w = corner_nd(D, v, frac, c, vc);
+                uint32_t h = oracle_hash_nd(D, vc) & mask;
+                for (int f = 0; f < F; ++f)
+                    dtable[((size_t)l * T + h) * F + f] += w * (double)g[(size_t)p * L * F + (size_t)l * F + f];
+            }
+        }
+}
+
+/* dL/dx_i = sum_l N_l sum_c (sum_f g e_c[f]) (d_i ? +1 : -1) prod_{j != i} (d_j ? frac_j : 1 - frac_j) */
+void oracle_backward_x_nd(int D, int L, int F, int log2T, const int *res, int dtype, const void *table,
+                          const float *x, const float *g, int64_t N, double *dx, int nthreads)
+{
+    size_t T = (size_t)1 << log2T;
+    uint32_t mask = (uint32_t)(T - 1);
+    int nc = 1 << D;
+    if (nthreads < 1)
+        nthreads = 1;
+#pragma omp parallel for schedule(static) num_threads(nthreads)
+    for (int64_t p = 0; p < N; ++p) {
+        double acc[7] = {0, 0, 0, 0, 0, 0, 0};
+        for (int l = 0; l < L; ++l) {
+            int64_t v[7], vc[7];
+            double frac[7];
+            locate_nd(D, x + (size_t)D * p, res[l], v, frac);
+            for (int c = 0; c < nc; ++c) {
+                (void)corner_nd(D, v, frac, c, vc);
+                uint32_t h = oracle_hash_nd(D, vc) & mask;
+                double ge = 0.0;
+                for (int f = 0; f < F; ++f)
+                    ge += (double)g[(size_t)p * L * F + (size_t)l * F + f] *
+                          table_value(table, dtype, ((size_t)l * T + h) * F + f);
+                for (int i = 0; i < D; ++i) {
+                    double dw = (double)res[l] * (((c >> i) & 1) ? 1.0 : -1.0);
+                    for (int j = 0; j < D; ++j)
+                        if (j != i)
+                            dw *= ((c >> j) & 1) ? frac[j] : 1.0 - frac[j];
+                    acc[i] += ge * dw;
+                }
+            }
+        }
+        for (int i = 0; i < D; ++i)
+            dx[(size_t)D * p + i] = acc[i];
+    }
+}

@@ -97,6 +97,22 @@ def test_create_rejects_invalid(args):
     assert e.value.code == hg.HASHGRID_ERR_ARG
 
 
+def test_create_nd():
+    for D in (2, 3, 4):
+        h = hg.hashgrid_create_nd(D, 8, 2, 12, 4, 128)
+        try:
+            assert hg.hashgrid_dims(h) == D
+            assert hg.hashgrid_resolutions(h) == oracle.resolutions(8, 4, 128)
+        finally:
+            hg.hashgrid_destroy(h)
+    assert hg.hashgrid_dims(hg.hashgrid_create(4, 2, 10, 2, 16)) == 3
+    for D in (0, 1, 5, 7):
+        h = ctypes.c_void_p(99)
+        assert hg.lib.hashgrid_create_nd(D, 8, 2, 12, 4, 128, 0, ctypes.byref(h)) == hg.HASHGRID_ERR_ARG
+        assert h.value is None
+    assert hg.hashgrid_dims(0) == 0
+
+
 def test_options():
     h = hg.hashgrid_create(16, 2, 19, 16, 512)
     try:

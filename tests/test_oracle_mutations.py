@@ -32,19 +32,37 @@ MUTATIONS = {
                               "double dw = 1.0 * (((c >> i) & 1) ? 1.0 : -1.0);"),
     "adam_no_bias_correction": ("double mhat = m[i] / c1;", "double mhat = m[i];"),
     "adam_not_sparse": ("        if (g == 0.0)\n            continue;\n        m[i]", "        m[i]"),
+    "nd_fourth_prime": ("2654435761u, 805459861u, 3674653429u,", "2654435761u, 805459861u, 3674653427u,"),
     "int64_hash_low_bits_lost": ("return (u0 * ORACLE_PRIME_X) ^ (u1 * ORACLE_PRIME_Y) ^ (u2 * ORACLE_PRIME_Z);",
                                  "return ((u0 * ORACLE_PRIME_X) ^ (u1 * ORACLE_PRIME_Y) ^ (u2 * ORACLE_PRIME_Z)) & 0x7fffffffu;"),
 }
 
-PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+def _pin_calls():
+    """Every pin as (name, function, kwargs), parametrized pins expanded."""
+    calls = []
+    for name in dir(pins):
+        if not name.startswith("test_"):
+            continue
+        fn = getattr(pins, name)
+        marks = [m for m in getattr(fn, "pytestmark", []) if m.name == "parametrize"]
+        if not marks:
+            calls.append((name, fn, {}))
+            continue
+        argname, values = marks[0].args[0], marks[0].args[1]
+        for v in values:
+            calls.append((name, fn, {argname: v}))
+    return calls
+
+
+PIN_TESTS = _pin_calls()
 
 
 def build_mutant(tmp_path, name):
     src = open(SRC).read()
     old, new = MUTATIONS[name]
-    assert src.count(old) == 1, f"mutation {name} does not apply"
+    assert src.count(old) >= 1, f"mutation {name} does not apply"
     path = tmp_path / f"{name}.c"
-    path.write_text(src.replace(old, new))
+    path.write_text(src.replace(old, new, 1))   # first occurrence: the 3-D function
     lib = tmp_path / f"lib_{name}.so"
     subprocess.run(["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
                     "-o", str(lib), str(path), "-lm"], check=True)
@@ -58,14 +76,16 @@ def test_pins_catch_mutation(tmp_path, name, monkeypatch):
     good = oracle._lib()                      # typed prototypes of the real library
     mut = ctypes.CDLL(path)
     for fn in ("oracle_resolutions", "oracle_hash3", "oracle_half_to_double", "oracle_indices",
-               "oracle_forward", "oracle_backward", "oracle_backward_x", "oracle_adam_step"):
+               "oracle_forward", "oracle_backward", "oracle_backward_x", "oracle_adam_step",
+               "oracle_hash_nd", "oracle_indices_nd", "oracle_forward_nd", "oracle_backward_nd", "oracle_backward_x_nd",
+               "oracle_bf16_to_double", "oracle_mlp_forward"):
         getattr(mut, fn).argtypes = getattr(good, fn).argtypes
         getattr(mut, fn).restype = getattr(good, fn).restype
     monkeypatch.setattr(oracle, "_LIB", mut)
     failed = []
-    for t in PIN_TESTS:
+    for name, fn, kwargs in PIN_TESTS:
         try:
-            t()
+            fn(**kwargs)
         except (AssertionError, ValueError):
-            failed.append(t.__name__)
+            failed.append(name)
     assert failed, f"mutation {name} passed every pin"

@@ -490,7 +490,8 @@ def bf16_values(bits):
 def test_bf16_decode():
     bits = np.arange(0, 65536, 97, dtype=np.uint32).astype(np.uint16)
     for b in bits:
-        want = bf16_values(np.array([b]))[0]
+        with np.errstate(invalid="ignore"):          # NaN patterns
+            want = bf16_values(np.array([b]))[0]
         got = oracle.bf16_to_double(int(b))
         assert (got == want) or (np.isnan(got) and np.isnan(want))
 
@@ -513,3 +514,94 @@ def test_mlp_matches_numpy_matmuls():
     want = a2 @ bf16_values(w3).T + b3.astype(np.float64)
     np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
     assert np.any(a1 == 0) and np.any(a1 > 0)           # ReLU active on both sides
+
+
+# ---------------------------------------------------------------------------------------
+# D-dimensional inputs (2^D corners; primes of Repro-HG sections 2.2 and 3)
+# ---------------------------------------------------------------------------------------
+
+PRIMES7 = (1, 2654435761, 805459861, 3674653429, 2097192037, 1434869437, 2165219737)
+
+
+def bigint_hash_nd(c, T=None):
+    h = 0
+    for ci, pi in zip(c, PRIMES7):
+        h ^= (int(ci) % 2**32) * pi
+    h %= 2**32
+    return h if T is None else h % T
+
+
+def test_hash_nd_bigint_and_primes():
+    rng = np.random.default_rng(90)
+    for D in range(1, 8):
+        for c in rng.integers(-2**33, 2**33, size=(200, D)):
+            assert oracle.hash_nd(c) == bigint_hash_nd(c)
+        for i in range(D):        # unit vectors give the primes themselves
+            e = np.zeros(D, dtype=np.int64)
+            e[i] = 1
+            assert oracle.hash_nd(e) == PRIMES7[i]
+    assert oracle.hash_nd([1, 1, 1, 1]) == 1 ^ 2654435761 ^ 805459861 ^ 3674653429
+
+
+def test_nd_at_three_dimensions_equals_3d_oracle():
+    g3, gn = Grid(4, 2, 10, 2, 16), oracle.GridND(3, 4, 2, 10, 2, 16)
+    rng = np.random.default_rng(91)
+    x = rng.random((300, 3), dtype=np.float32)
+    t = rng.standard_normal((4, 1024, 2)).astype(np.float32)
+    up = rng.standard_normal((300, 8)).astype(np.float32)
+    np.testing.assert_array_equal(gn.indices(x), g3.indices(x))
+    np.testing.assert_array_equal(gn.forward(x, t), g3.forward(x, t))
+    np.testing.assert_array_equal(gn.backward(x, up), g3.backward(x, up))
+    np.testing.assert_array_equal(gn.backward_x(x, t, up), g3.backward_x(x, t, up))
+
+
+def hat_basis_nd(x, table, res, T):
+    N, D = x.shape
+    L, _, F = table.shape
+    out = np.zeros((N, L * F))
+    for p in range(N):
+        for l, n in enumerate(res):
+            xs = [float(np.float32(x[p, i]) * np.float32(n)) for i in range(D)]
+            base = [int(np.floor(v)) for v in xs]
+            for off in np.ndindex(*([4] * D)):
+                v = [base[i] - 1 + off[i] for i in range(D)]
+                w = 1.0
+                for i in range(D):
+                    w *= max(0.0, 1 - abs(xs[i] - v[i]))
+                if w:
+                    out[p, l * F:(l + 1) * F] += w * table[l, bigint_hash_nd(v, T)].astype(np.float64)
+    return out
+
+
+@pytest.mark.parametrize("D", [2, 4])
+def test_nd_forward_hat_basis_and_weight_sum(D):
+    g = oracle.GridND(D, 3, 2, 10, 2, 8)
+    rng = np.random.default_rng(92 + D)
+    t = rng.standard_normal((3, 1024, 2)).astype(np.float32)
+    x = rng.random((40, D), dtype=np.float32)
+    x[0] = np.float32(1.0)
+    x[1] = np.float32(0.0)
+    np.testing.assert_allclose(g.forward(x, t), hat_basis_nd(x, t, g.res, g.T), rtol=0, atol=1e-12)
+    ones = g.forward(x, np.ones((3, 1024, 2), dtype=np.float32))
+    assert np.max(np.abs(ones - 1.0)) <= 8 * np.finfo(np.float64).eps
+
+
+@pytest.mark.parametrize("D", [2, 4])
+def test_nd_backward_adjoint_and_input_gradient(D):
+    g = oracle.GridND(D, 4, 2, 10, 2, 16)
+    rng = np.random.default_rng(95 + D)
+    t = rng.standard_normal((4, 1024, 2)).astype(np.float32)
+    up = rng.standard_normal((60, 8)).astype(np.float32)
+    k = rng.integers(0, 32, size=(60, D))
+    x = ((k + 0.5) / 32.0).astype(np.float32)
+    lhs = float(np.sum(up.astype(np.float64) * g.forward(x, t)))
+    rhs = float(np.sum(g.backward(x, up) * t.astype(np.float64)))
+    assert abs(lhs - rhs) <= 1e-12 * max(abs(lhs), 1.0)
+    dx = g.backward_x(x, t, up)
+    h = np.float32(2.0 ** -12)
+    for i in range(D):
+        xp, xm = x.copy(), x.copy()
+        xp[:, i] += h
+        xm[:, i] -= h
+        fd = np.sum(up.astype(np.float64) * (g.forward(xp, t) - g.forward(xm, t)), axis=1) / (2 * float(h))
+        np.testing.assert_allclose(dx[:, i], fd, rtol=1e-9, atol=1e-9)

@@ -606,3 +606,53 @@ def test_backward_half_widths(F):
     hg.hashgrid_backward_half(grid.handle, dev(x), dev(g), 2000, d)
     torch.cuda.synchronize()
     check_half_gradient(og, x, g, d.cpu().numpy())
+
+
+# ---------------------------------------------------------------------------------------
+# D-dimensional inputs
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("F", [1, 2, 4, 8])
+@pytest.mark.parametrize("D", [2, 4])
+def test_nd_parity(D, F):
+    """Indices bit-exact, forward within 1e-6 of sum_c w_c |e_c| (2^D products of D-1
+    fp32 roundings and 2^D fma: ~(D + 2^D) ulp), fp32 and fp16 gradients, and dL/dx, for
+    D = 2 and 4 against the oracle's D-dimensional functions."""
+    hg = hgmod()
+    L, log2T = 6, 12
+    grid = hg.HashGrid(L, F, log2T, 3, 150, D=D)
+    og = oracle.GridND(D, L, F, log2T, 3, 150)
+    rng = np.random.default_rng(100 + 10 * D + F)
+    table = workloads.table_values(rng, L, 2**log2T, F)
+    x = rng.random((2000 + 37, D), dtype=np.float32)
+    x[:4] = np.float32(1.0)
+    x[4:8] = -rng.random((4, D), dtype=np.float32)
+    g = workloads.upstream_grads(rng, x.shape[0], L * F)
+    x_d, t_d, g_d = dev(x), dev(table), dev(g)
+    np.testing.assert_array_equal(grid.indices(x_d).cpu().numpy().view(np.uint32), og.indices(x))
+    out = grid.forward(x_d, t_d).cpu().numpy().astype(np.float64)
+    ref = og.forward(x, table, nthreads=THREADS)
+    bound = og.forward(x, np.abs(table), nthreads=THREADS)
+    assert np.all(np.abs(out - ref) <= 1e-6 * bound + 1e-30)
+    dref = og.backward(x, g, nthreads=THREADS)
+    assert rel_l2(grid.backward(x_d, g_d).cpu().numpy(), dref) <= BWD_REL_L2
+    dh = torch.zeros((L, 2**log2T, F), dtype=torch.float16, device="cuda")
+    hg.hashgrid_backward_half(grid.handle, x_d, g_d, x.shape[0], dh)
+    torch.cuda.synchronize()
+    assert rel_l2(dh.cpu().numpy(), dref) <= 2e-2
+    dx = grid.backward_input(x_d, g_d, t_d).cpu().numpy().astype(np.float64)
+    dxref = og.backward_x(x, table, g, nthreads=THREADS)
+    tmax = float(np.max(np.abs(table)))
+    B = np.zeros(x.shape[0])
+    for l, n in enumerate(og.res):
+        B += float(n) * 2.0 * np.sum(np.abs(g[:, l * F:(l + 1) * F].astype(np.float64)), axis=1) * tmax
+    assert np.all(np.abs(dx - dxref) <= 1e-5 * B[:, None] * 2 ** (D - 3) + 1e-30)
+
+
+def test_nd_mlp_rejected():
+    hg = hgmod()
+    grid = hg.HashGrid(16, 2, 12, 16, 512, D=2)
+    z = torch.zeros(64 * 64, device="cuda")
+    rc = hg.lib.hashgrid_mlp_forward(grid.handle, z.data_ptr(), 4, z.data_ptr(), z.data_ptr(), z.data_ptr(),
+                                     z.data_ptr(), z.data_ptr(), z.data_ptr(), z.data_ptr(), z.data_ptr(), None, None)
+    assert rc == hg.HASHGRID_ERR_ARG
