@@ -41,8 +41,10 @@
  *     any launch and nothing is written. A failed launch returns HASHGRID_ERR_CUDA.
  *     hashgrid_last_error() gives a message for the last failure on the calling thread.
  *   - N = 0 is a valid no-op (returns HASHGRID_OK, pointers may be NULL).
- *   - A handle may be used from several threads and streams at once; it is read-only after
- *     hashgrid_create.
+ *   - A handle may be used from several threads and streams at once; set its options before
+ *     sharing it (hashgrid_set_option is not synchronised with running calls).
+ *   - The compute calls may be captured into CUDA graphs: their host-side checks only query
+ *     pointer attributes, and each call is a single kernel launch on cuda_stream.
  */
 #ifndef HASHGRID_H
 #define HASHGRID_H
