@@ -3,14 +3,17 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
                     [--workload NAME] [--skip-cpu-baseline] [--skip-e2e] [--skip-fwd-leg]
+                    [--skip-next-rows]
 
 One step = one pass of the whole hot path over one batch resident in HBM: zero the table
 gradient, forward (voxel, 8 corner hashes, gathers, trilinear interpolation, level-major
 output rows), backward (weighted scatter-add into the fp32 gradient table). The default
 workload is the 16-level, F=2, T=2^19 grid (N 16->512) on 2^14 rays x 64 stratified
 samples (2^20 points); the forward-only leg on 2^18 uniform points of the same grid is
-reported under "fwd". L2 is flushed (256 MiB write) before every timed step, outside the
-step's events. Rank 0 prints one JSON line.
+reported under "fwd", and the gradient w.r.t. x, a sparse Adam step, the encoding fused with
+the MLP and the fp16-gradient backward on the same batch under "next_rows". L2 is flushed
+(256 MiB write) before every timed step, outside the step's events. Rank 0 prints one JSON
+line.
 
 Multi-GPU: one process per GPU (torchrun); every rank encodes its own batch with its own
 table replica (points are independent), there is no collective on the data path, and the
@@ -368,6 +371,96 @@ def time_e2e(res: Resident, steps: int, warmup: int, device) -> dict:
     return {"ms": ms, "h2d": h2d, "d2h": d2h}
 
 
+def time_launches(fn, steps: int, warmup: int, device, before=None) -> float:
+    """Mean milliseconds of ``fn`` (one launch on the current stream) over ``steps`` timed
+    calls, each after an L2 flush and the optional untimed ``before``."""
+    import torch
+    stream = torch.cuda.current_stream(device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    for _ in range(warmup):
+        if before is not None:
+            before()
+        fn()
+    ts = []
+    for _ in range(steps):
+        flush.fill_(1)
+        if before is not None:
+            before()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        ts.append((a, b))
+    torch.cuda.synchronize(device)
+    return statistics.mean(a.elapsed_time(b) for a, b in ts)
+
+
+def time_next_rows(res: Resident, steps: int, warmup: int, device) -> tuple[dict, int]:
+    """The operations beyond the forward/backward pair, on the same resident batch: the
+    gradient w.r.t. x, one sparse Adam step over the table, the encoding fused with the
+    3-layer MLP on the tensor cores, and the backward into an fp16 gradient table. Each is
+    one launch, timed alone. Returns the JSON object and the number of timed launches."""
+    import torch
+    hg, w, N, sp = res.hg, res.w, res.N, torch.cuda.current_stream(device).cuda_stream
+    peak, src = measured_peaks()
+    s = 2 if w.dtype == "f16" else 4
+    LF = w.L * w.F
+    out, launches = {"workload": w.name, "peak_note": f"{src} HBM peak"}, 0
+
+    def entry(ms, nbytes, **extra):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": round(ms, 5), "points_per_s": round(N / (ms * 1e-3), 1),
+                "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                             "frac": round(gbs / peak, 4), "bytes_per_launch": int(nbytes)}, **extra}
+
+    # dL/dx: x, upstream gradient and 8 corner gathers per level in; dL/dx out.
+    dx = torch.empty((N, 3), dtype=torch.float32, device=device)
+    ms = time_launches(lambda: hg.hashgrid_backward_input(res.handle, res.x, res.g, N, res.table, dx, sp),
+                       steps, warmup, device)
+    out["backward_input"] = entry(ms, N * (12 + 4 * LF + 8 * LF * s + 12))
+    launches += steps
+
+    # Sparse Adam over the table with the gradient of one backward pass: every gradient
+    # element is read; parameter, m and v are read and written where the gradient is nonzero.
+    if w.dtype == "f32":
+        res.dtable.zero_()
+        res.backward_pass(sp)
+        nnz = int(torch.count_nonzero(res.dtable))
+        table, m, v = res.table.clone(), torch.zeros_like(res.table), torch.zeros_like(res.table)
+        step = [0]
+
+        def adam():
+            step[0] += 1
+            hg.hashgrid_adam_step(res.handle, table, m, v, res.dtable, step[0], 1e-2, zero_grad=False, stream=sp)
+        ms = time_launches(adam, steps, warmup, device)
+        out["adam_step"] = entry(ms, 4 * res.dtable.numel() + 24 * nnz, elements=res.dtable.numel(), nonzero=nnz)
+        out["adam_step"].pop("points_per_s")
+        launches += steps
+        del table, m, v
+
+    # Encoding + MLP (LF -> 64 -> 64 -> 4, bf16 operands, fp32 accumulation): x and the
+    # gathers in, 4 outputs per point out; the weights stay in shared memory.
+    if LF in (16, 32, 48, 64):
+        gen = torch.Generator(device="cpu").manual_seed(7)
+        bf = lambda *shape: (torch.randn(*shape, generator=gen) * 0.1).to(torch.bfloat16).to(device)  # noqa: E731
+        w1, w2, w3 = bf(64, LF), bf(64, 64), bf(4, 64)
+        b1, b2, b3 = (torch.zeros(64, device=device), torch.zeros(64, device=device), torch.zeros(4, device=device))
+        y = torch.empty((N, 4), dtype=torch.float32, device=device)
+        ms = time_launches(lambda: hg.hashgrid_mlp_forward(res.handle, res.x, N, res.table, w1, b1, w2, b2, w3, b3, y,
+                                                           stream=sp), steps, warmup, device)
+        flops = 2 * N * (LF * 64 + 64 * 64 + 64 * 4)
+        out["mlp_forward"] = entry(ms, N * (12 + 8 * LF * s + 16), tensor_tflops=round(flops / (ms * 1e-3) / 1e12, 2))
+        launches += steps
+
+    # Backward into an fp16 gradient table (packed f16x2 reductions), zeroed before each call.
+    dh = torch.zeros((w.L, w.T, w.F), dtype=torch.float16, device=device)
+    ms = time_launches(lambda: hg.hashgrid_backward_half(res.handle, res.x, res.g, N, dh, sp), steps, warmup,
+                       device, before=dh.zero_)
+    out["backward_half"] = entry(ms, N * (12 + 4 * LF + 8 * LF * 2))
+    launches += steps
+    return out, launches
+
+
 def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, kernel: str) -> dict:
     peak, src = measured_peaks()
     bytes_per_launch = algorithmic_bytes_per_point(w, kind) * points
@@ -504,6 +597,10 @@ def run_b200(args) -> None:
         fres.close()
         del fres
 
+    if not args.skip_next_rows and w.backward:
+        line["next_rows"], n = time_next_rows(res, min(args.steps, 20), min(args.warmup, 3), device)
+        launches += n
+
     if not args.skip_e2e:
         e = time_e2e(res, args.steps, min(args.warmup, 3), device)
         launches += args.steps * (2 if w.backward else 1)
@@ -536,6 +633,8 @@ def main(argv=None) -> None:
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-fwd-leg", action="store_true")
+    ap.add_argument("--skip-next-rows", action="store_true",
+                    help="skip timing dL/dx, Adam, the fused MLP and the fp16-gradient backward")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "b200":
         print("note: fewer than 3 warm-up steps; the timing rules want at least 3", file=sys.stderr)

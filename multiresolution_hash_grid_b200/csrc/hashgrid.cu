@@ -9,6 +9,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -291,18 +292,21 @@ int launch_mlp_forward(const hashgrid_s* h, const float* x, int64_t N, const voi
                        const float* b1, const void* w2, const float* b2, const void* w3, const float* b3, float* y,
                        int* status, cudaStream_t s) {
     auto k = hg::mlp::mlp_forward_kernel<F, TT, K1>;
-    const size_t smem = hg::mlp::smem_bytes(K1);
+    const size_t smem = hg::mlp::ws_smem_bytes(K1);
     if (int rc = prepare_smem(k, smem)) return rc;
-    int dev = 0, sms = 148;
+    int dev = 0, sms = 148, smem_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // Persistent grid: as many CTAs as fit per SM (registers and shared memory allow 3 for
-    // F <= 4, 2 for F = 8; TMEM holds 3 x 64 columns of 512). More would only queue.
-    const int per_sm = F == 8 ? 2 : 3;
+    cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    // Persistent grid: as many CTAs as fit per SM (registers allow 2; shared memory as
+    // computed, with the 1 KB the runtime reserves per CTA). More would only queue behind the
+    // resident ones.
+    const int fit = (int)((size_t)smem_sm / (smem + 1024));
+    const int per_sm = std::max(1, std::min(hg::mlp::kCtasPerSm, fit));
     const int64_t tiles = (N + hg::mlp::kM - 1) / hg::mlp::kM;
     const int64_t cap = (int64_t)sms * per_sm;
     const unsigned blocks = (unsigned)(tiles < cap ? tiles : cap);
-    k<<<blocks, hg::mlp::kThreads, smem, s>>>(h->lp, x, N, static_cast<const TT*>(table),
+    k<<<blocks, hg::mlp::block_threads(F), smem, s>>>(h->lp, x, N, static_cast<const TT*>(table),
                                                static_cast<const uint16_t*>(w1), b1, static_cast<const uint16_t*>(w2),
                                                b2, static_cast<const uint16_t*>(w3), b3, y, status);
     return launch_status("mlp_forward");
