@@ -407,17 +407,18 @@ def time_next_rows(res: Resident, steps: int, warmup: int, device) -> tuple[dict
     LF = w.L * w.F
     out, launches = {"workload": w.name, "peak_note": f"{src} HBM peak"}, 0
 
-    def entry(ms, nbytes, **extra):
+    def entry(ms, nbytes, kernel, **extra):
         gbs = nbytes / (ms * 1e-3) / 1e9
         return {"ms": round(ms, 5), "points_per_s": round(N / (ms * 1e-3), 1),
-                "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                             "frac": round(gbs / peak, 4), "bytes_per_launch": int(nbytes)}, **extra}
+                "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(gbs, 1), "peak": peak,
+                             "unit": "GB/s", "frac": round(gbs / peak, 4), "bytes_per_launch": int(nbytes),
+                             "traffic": ncu_traffic(kernel, w.name)}, **extra}
 
     # dL/dx: x, upstream gradient and 8 corner gathers per level in; dL/dx out.
     dx = torch.empty((N, 3), dtype=torch.float32, device=device)
     ms = time_launches(lambda: hg.hashgrid_backward_input(res.handle, res.x, res.g, N, res.table, dx, sp),
                        steps, warmup, device)
-    out["backward_input"] = entry(ms, N * (12 + 4 * LF + 8 * LF * s + 12))
+    out["backward_input"] = entry(ms, N * (12 + 4 * LF + 8 * LF * s + 12), "backward_input_kernel")
     launches += steps
 
     # Sparse Adam over the table with the gradient of one backward pass: every gradient
@@ -433,7 +434,8 @@ def time_next_rows(res: Resident, steps: int, warmup: int, device) -> tuple[dict
             step[0] += 1
             hg.hashgrid_adam_step(res.handle, table, m, v, res.dtable, step[0], 1e-2, zero_grad=False, stream=sp)
         ms = time_launches(adam, steps, warmup, device)
-        out["adam_step"] = entry(ms, 4 * res.dtable.numel() + 24 * nnz, elements=res.dtable.numel(), nonzero=nnz)
+        out["adam_step"] = entry(ms, 4 * res.dtable.numel() + 24 * nnz, "adam_kernel", elements=res.dtable.numel(),
+                                 nonzero=nnz)
         out["adam_step"].pop("points_per_s")
         launches += steps
         del table, m, v
@@ -449,14 +451,15 @@ def time_next_rows(res: Resident, steps: int, warmup: int, device) -> tuple[dict
         ms = time_launches(lambda: hg.hashgrid_mlp_forward(res.handle, res.x, N, res.table, w1, b1, w2, b2, w3, b3, y,
                                                            stream=sp), steps, warmup, device)
         flops = 2 * N * (LF * 64 + 64 * 64 + 64 * 4)
-        out["mlp_forward"] = entry(ms, N * (12 + 8 * LF * s + 16), tensor_tflops=round(flops / (ms * 1e-3) / 1e12, 2))
+        out["mlp_forward"] = entry(ms, N * (12 + 8 * LF * s + 16), "mlp_forward_kernel",
+                                   tensor_tflops=round(flops / (ms * 1e-3) / 1e12, 2))
         launches += steps
 
     # Backward into an fp16 gradient table (packed f16x2 reductions), zeroed before each call.
     dh = torch.zeros((w.L, w.T, w.F), dtype=torch.float16, device=device)
     ms = time_launches(lambda: hg.hashgrid_backward_half(res.handle, res.x, res.g, N, dh, sp), steps, warmup,
                        device, before=dh.zero_)
-    out["backward_half"] = entry(ms, N * (12 + 4 * LF + 8 * LF * 2))
+    out["backward_half"] = entry(ms, N * (12 + 4 * LF + 8 * LF * 2), "backward_kernel_half")
     launches += steps
     return out, launches
 

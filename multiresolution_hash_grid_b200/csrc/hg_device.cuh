@@ -1053,15 +1053,16 @@ __global__ void __launch_bounds__(kLevelBlock) backward_kernel_runs_levels(Level
 // d frac_i / d x_i = N_l, so with s_c = sum_f g_f e_c[f]:
 //   dL/dx_i = sum_l N_l * sum_c s_c * (d_i ? +1 : -1) * prod_{j != i} (d_j ? frac_j : 1 - frac_j).
 // Point-major: a block stages its x and upstream-gradient rows, each (point, level) thread
-// gathers the 8 corners and writes its 3 partials to shared memory as [level][axis][point]
-// (conflict-free), then one thread per point sums its levels in order and stores dL/dx.
+// gathers the 8 corners and writes its 3 partials to shared memory as [level][point][axis]
+// (stride 3 across lanes: conflict-free), then one thread per (point, axis) sums the levels
+// in order (consecutive words across lanes) and stores dL/dx.
 // ---------------------------------------------------------------------------------------
 __host__ __device__ constexpr size_t input_grad_smem_bytes(int BP, int L, int F) {
     return tile_smem_bytes(BP, L, F) + sizeof(float) * (size_t)BP * L * 3;
 }
 
 template <int F, typename TT, int BP>
-__global__ void __launch_bounds__(512, 2) backward_input_kernel(LevelParams lp, const float* __restrict__ x,
+__global__ void __launch_bounds__(512, F <= 2 ? 3 : 2) backward_input_kernel(LevelParams lp, const float* __restrict__ x,
                                                                 const float* __restrict__ dout, int64_t N,
                                                                 const TT* __restrict__ table,
                                                                 float* __restrict__ dx) {
@@ -1071,7 +1072,7 @@ __global__ void __launch_bounds__(512, 2) backward_input_kernel(LevelParams lp, 
     const int S = W + row_pad(F);
     float* xs = smem;
     float* gs = smem + BP * 3;
-    float* part = gs + BP * S;  // [L][3][BP]
+    float* part = gs + BP * S;  // [L][BP][3]
     const int64_t p0 = (int64_t)blockIdx.x * BP;
     const int nvalid = (int)min((int64_t)BP, N - p0);
 
@@ -1117,16 +1118,16 @@ __global__ void __launch_bounds__(512, 2) backward_input_kernel(LevelParams lp, 
                 d2 = fmaf(s2, w0[b0] * w1[b1], d2);
             }
             const float n = lp.scale[l];
-            part[(l * 3 + 0) * BP + pl] = n * d0;
-            part[(l * 3 + 1) * BP + pl] = n * d1;
-            part[(l * 3 + 2) * BP + pl] = n * d2;
+            float* pp = part + ((size_t)l * BP + pl) * 3;  // stride 3 across lanes: conflict-free
+            pp[0] = n * d0;
+            pp[1] = n * d1;
+            pp[2] = n * d2;
         }
     }
     __syncthreads();
-    for (int t = threadIdx.x; t < nvalid * 3; t += blockDim.x) {
-        const int pt = t / 3, i = t - 3 * (t / 3);
+    for (int t = threadIdx.x; t < nvalid * 3; t += blockDim.x) {  // t = 3 * point + axis
         float s = 0.f;
-        for (int l = 0; l < L; ++l) s += part[(l * 3 + i) * BP + pt];
+        for (int l = 0; l < L; ++l) s += part[(size_t)l * BP * 3 + t];
         __stcs(dx + p0 * 3 + t, s);
     }
 }
