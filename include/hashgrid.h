@@ -236,8 +236,9 @@ int hashgrid_adam_step(hashgrid_t h, void *table, float *adam_m, float *adam_v, 
  * w3: [4][64] bf16 (uint16 bit patterns), row-major [out][in] like a torch Linear weight;
  * b1: [64], b2: [64], b3: [4] fp32; y: [N,4] fp32 (overwritten). L*F must be 16, 32, 48
  * or 64 (HASHGRID_ERR_ARG otherwise). device_status: NULL or a device int the caller sets
- * to 0; the kernel sets it to 1 if it gave up waiting for the tensor cores (it then stops
- * early and y is incomplete).
+ * to 0; the kernel sets it to 1 if a bounded wait inside it ran out (on the tensor cores'
+ * completion or on the hand-off between its encoding and MMA warps); it then stops early
+ * and y is incomplete.
  */
 int hashgrid_mlp_forward(hashgrid_t h, const float *x, int64_t N, const void *table, const void *w1,
                          const float *b1, const void *w2, const float *b2, const void *w3,
