@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(block_threads(F), kCtasPerSm) mlp_forward_kern
                     Corners cr;
                     locate_corners(x0, x1, x2, lp.scale[l], lp.mask, cr);
                     float e[8][F];
-                    gather_corners<F, TT, kGatherCorner>(table + (uint64_t)l * lp.T * F, cr, e);
+                    gather_corners<F, TT, kGatherCorner, std::is_same<TT, float>::value>(table + (uint64_t)l * lp.T * F, cr, e);
 #pragma unroll
                     for (int f = 0; f < F; ++f) {
                         float acc = cr.w[0] * e[0][f];
