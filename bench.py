@@ -51,6 +51,7 @@ FWD_WORKLOAD = "grid_L16F2T19"
 FLUSH_BYTES = 256 << 20
 CPU_SAMPLE_POINTS = 1 << 18
 REFERENCE_SAMPLE_POINTS = 1 << 15
+NEXT_ROWS_CPU_SAMPLE = 1 << 16
 FALLBACK_HBM_GBS = 6650.0
 GATHER_MODES = {"auto": 0, "corner": 1, "sector": 2, "pair": 3}  # HASHGRID_GATHER_*
 SCHEDULES = {"auto": 0, "point": 1, "level": 2}             # HASHGRID_SCHEDULE_*
@@ -435,7 +436,7 @@ def time_next_rows(res: Resident, steps: int, warmup: int, device) -> tuple[dict
             hg.hashgrid_adam_step(res.handle, table, m, v, res.dtable, step[0], 1e-2, zero_grad=False, stream=sp)
         ms = time_launches(adam, steps, warmup, device)
         out["adam_step"] = entry(ms, 4 * res.dtable.numel() + 24 * nnz, "adam_kernel", elements=res.dtable.numel(),
-                                 nonzero=nnz)
+                                 nonzero=nnz, elements_per_s=round(res.dtable.numel() / (ms * 1e-3), 1))
         out["adam_step"].pop("points_per_s")
         launches += steps
         del table, m, v
@@ -498,6 +499,57 @@ def cpu_baseline(w: workloads.Workload, sample: int, budget_s: float = 10.0) -> 
             "sample": f"{passes} passes over the first {n} points of {w.name} (seed {rank_seed(0)}), "
                       f"{'fwd+bwd' if w.backward else 'fwd'}; fwd parallel over points, "
                       f"bwd over the {w.L} levels; {dt:.1f} s"}
+
+
+def cpu_next_rows(w: workloads.Workload, sample: int, budget_s: float = 3.0) -> dict:
+    """The oracle's counterparts of the next-row kernels, as they stand, on the host cores:
+    dL/dx and the encoding + MLP over a sample of the workload's points, and sparse Adam
+    over the whole table with the oracle's own gradient of that sample (computed untimed),
+    each repeated for about ``budget_s`` seconds."""
+    import oracle
+    threads = oracle.default_threads()
+    inp = workloads.make_inputs(w, seed=rank_seed(0), n_points=sample, grads=True)
+    og = oracle.Grid(w.L, w.F, w.log2T, w.N_min, w.N_max, oracle.F16 if w.dtype == "f16" else oracle.F32)
+    n = inp.x.shape[0]
+
+    def rate(fn):
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            fn()
+            reps += 1
+            dt = time.perf_counter() - t0
+            if dt >= budget_s:
+                return reps, dt
+
+    out = {"cores": threads, "kind": "oracle"}
+    reps, dt = rate(lambda: og.backward_x(inp.x, inp.table, inp.g, nthreads=threads))
+    out["backward_input"] = {"value": round(n * reps / dt, 1), "unit": UNIT,
+                             "sample": f"{reps} passes over the first {n} points, parallel over points"}
+    LF = w.L * w.F
+    if LF in (16, 32, 48, 64):
+        rng = np.random.default_rng(7)
+        bf = lambda *shape: (rng.standard_normal(shape).astype(np.float32) * 0.1).view(np.uint32) >> 16  # noqa: E731
+        w1, w2, w3 = bf(64, LF).astype(np.uint16), bf(64, 64).astype(np.uint16), bf(4, 64).astype(np.uint16)
+        b = np.zeros(64, dtype=np.float32)
+        reps, dt = rate(lambda: og.mlp_forward(inp.x, inp.table, w1, b, w2, b, w3, b[:4], nthreads=threads))
+        out["mlp_forward"] = {"value": round(n * reps / dt, 1), "unit": UNIT,
+                              "sample": f"{reps} passes over the first {n} points, parallel over points"}
+    if w.dtype == "f32":
+        # one level's slice of the table (the oracle's step is elementwise, so its rate per
+        # element does not depend on which slice)
+        grad = og.backward(inp.x, inp.g, levels=(w.L - 1, w.L), nthreads=threads)[w.L - 1].astype(np.float32)
+        table = inp.table[w.L - 1]
+        m, v = np.zeros_like(grad), np.zeros_like(grad)
+        step = [0]
+
+        def adam():
+            step[0] += 1
+            oracle.adam_step(table, m, v, grad, step[0], 1e-2)
+        reps, dt = rate(adam)
+        out["adam_step"] = {"value": round(grad.size * reps / dt, 1), "unit": "elements/s",
+                            "sample": f"{reps} steps over the finest level's {grad.size} elements with the "
+                                      f"gradient of {n} points (single thread, fp64)"}
+    return out
 
 
 # ---------------------------------------------------------------------------------------
@@ -603,6 +655,8 @@ def run_b200(args) -> None:
     if not args.skip_next_rows and w.backward:
         line["next_rows"], n = time_next_rows(res, min(args.steps, 20), min(args.warmup, 3), device)
         launches += n
+        if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+            line["next_rows"]["cpu_oracle"] = cpu_next_rows(w, min(NEXT_ROWS_CPU_SAMPLE, res.N))
 
     if not args.skip_e2e:
         e = time_e2e(res, args.steps, min(args.warmup, 3), device)

@@ -69,3 +69,14 @@ def test_single_process_helpers():
     assert bench.algorithmic_bytes_per_point(w, "bwd") == 1164
     assert bench.algorithmic_bytes_per_point(workloads.WORKLOADS["half_L16F2T19"], "fwdbwd") == 1816
     assert bench.algorithmic_bytes_per_point(workloads.WORKLOADS["large_L16F4T22"], "fwdbwd") == 4632
+
+
+def test_cpu_oracle_timers():
+    # the bench's CPU legs run the oracle as it stands on a bounded sample
+    w = workloads.WORKLOADS["tiny_L4F2T10"]
+    base = bench.cpu_baseline(w, 512, budget_s=0.05)
+    assert base["kind"] == "oracle" and base["value"] > 0 and base["cores"] >= 1
+    rows = bench.cpu_next_rows(w, 512, budget_s=0.05)
+    assert rows["backward_input"]["value"] > 0
+    assert rows["adam_step"]["value"] > 0 and rows["adam_step"]["unit"] == "elements/s"
+    assert "mlp_forward" not in rows   # L*F = 8 has no MLP
