@@ -553,6 +553,63 @@ def test_mlp_forward_full_size_sampled():
     check_mlp(og, inp.x[rows], table, wts, y.cpu().numpy()[rows])
 
 
+@pytest.mark.parametrize("N", [0, 1, 127, 128, 129, 3 * 2 * 148 * 128 + 77])
+def test_mlp_forward_tile_edges(N):
+    """Below, at and above one 128-point tile, and enough tiles that every persistent CTA
+    cycles both encoding buffers at least once (3+ tiles per CTA): every row against the
+    oracle; N = 0 writes nothing. Two calls give bit-identical results (no atomics)."""
+    hg = hgmod()
+    w = workloads.WORKLOADS["rays_L16F2T19"]
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max)
+    rng = np.random.default_rng(72)
+    table = (rng.standard_normal((w.L, w.T, w.F)) * 0.3).astype(np.float32)
+    x = workloads.ray_points(rng, (N + 63) // 64)[:N].astype(np.float32).reshape(-1, 3)
+    wts = mlp_weights(rng, 32)
+    y = torch.full((max(N, 1), 4), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    args = (dev(x) if N else torch.empty((1, 3), device="cuda"), N, dev(table), *[dev(v) for v in wts])
+    hg.hashgrid_mlp_forward(grid.handle, *args, y, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    if N == 0:
+        assert torch.isnan(y).all()
+        return
+    first = y.clone()
+    hg.hashgrid_mlp_forward(grid.handle, *args, y, status)
+    torch.cuda.synchronize()
+    assert torch.equal(first, y)
+    check_mlp(og, x, table, wts, y.cpu().numpy())
+
+
+def test_mlp_forward_graph_capture():
+    """The fused MLP captured in a CUDA graph and replayed equals the eager call bit for bit."""
+    hg = hgmod()
+    w = workloads.WORKLOADS["rays_L16F2T19"]
+    grid, _ = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max)
+    rng = np.random.default_rng(73)
+    table = dev((rng.standard_normal((w.L, w.T, w.F)) * 0.3).astype(np.float32))
+    x = dev(workloads.ray_points(rng, 300).astype(np.float32))
+    wts = [dev(v) for v in mlp_weights(rng, 32)]
+    N = x.shape[0]
+    eager = torch.empty((N, 4), device="cuda")
+    hg.hashgrid_mlp_forward(grid.handle, x, N, table, *wts, eager)
+    y = torch.empty((N, 4), device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        hg.hashgrid_mlp_forward(grid.handle, x, N, table, *wts, y, stream=s.cuda_stream)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    y.fill_(float("nan"))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        hg.hashgrid_mlp_forward(grid.handle, x, N, table, *wts, y, stream=s.cuda_stream)
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, eager)
+
+
 # ---------------------------------------------------------------------------------------
 # fp16 gradient tables (packed f16x2 reductions)
 # ---------------------------------------------------------------------------------------
