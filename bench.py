@@ -50,7 +50,7 @@ DEFAULT_WORKLOAD = "rays_L16F2T19"
 FWD_WORKLOAD = "grid_L16F2T19"
 FLUSH_BYTES = 256 << 20
 CPU_SAMPLE_POINTS = 1 << 18
-REFERENCE_SAMPLE_POINTS = 1 << 15
+REFERENCE_SAMPLE_POINTS = 1 << 17
 NEXT_ROWS_CPU_SAMPLE = 1 << 16
 FALLBACK_HBM_GBS = 6650.0
 GATHER_MODES = {"auto": 0, "corner": 1, "sector": 2, "pair": 3}  # HASHGRID_GATHER_*
@@ -570,9 +570,12 @@ def run_reference(args) -> None:
     inp = workloads.make_inputs(w, seed=rank_seed(0), n_points=REFERENCE_SAMPLE_POINTS, grads=True)
     og = oracle.Grid(w.L, w.F, w.log2T, w.N_min, w.N_max, oracle.F16 if w.dtype == "f16" else oracle.F32)
 
-    def step():
+    dtable = np.zeros((w.L, w.T, w.F))
+
+    def step():   # as in the GPU arm's step: forward, zero the gradient table, backward
         og.forward(inp.x, inp.table, nthreads=threads)
-        og.backward(inp.x, inp.g, nthreads=threads)
+        dtable.fill(0.0)
+        og.backward(inp.x, inp.g, nthreads=threads, dtable=dtable)
 
     for _ in range(args.warmup):
         step()
@@ -582,8 +585,8 @@ def run_reference(args) -> None:
     dt = time.perf_counter() - t0
     n = inp.x.shape[0]
     value = n * args.steps / dt
-    sample = (f"{n} points of {w.name} per step (seed {rank_seed(0)}), fwd+bwd; fwd parallel over "
-              f"points, bwd over the {w.L} levels")
+    sample = (f"{n} points of {w.name} per step (seed {rank_seed(0)}), fwd + zeroing of the fp64 gradient "
+              f"table + bwd; fwd parallel over points, bwd over the {w.L} levels")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
