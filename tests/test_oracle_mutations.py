@@ -35,6 +35,18 @@ MUTATIONS = {
     "nd_fourth_prime": ("2654435761u, 805459861u, 3674653429u,", "2654435761u, 805459861u, 3674653427u,"),
     "int64_hash_low_bits_lost": ("return (u0 * ORACLE_PRIME_X) ^ (u1 * ORACLE_PRIME_Y) ^ (u2 * ORACLE_PRIME_Z);",
                                  "return ((u0 * ORACLE_PRIME_X) ^ (u1 * ORACLE_PRIME_Y) ^ (u2 * ORACLE_PRIME_Z)) & 0x7fffffffu;"),
+    # the MLP and its bf16 weights
+    "mlp_missing_relu": ("            a1[o] = s > 0.0 ? s : 0.0;", "            a1[o] = s;"),
+    "mlp_bias_dropped": ("            double s = (double)b2[o];", "            double s = 0.0;"),
+    "mlp_w1_transposed": ("oracle_bf16_to_double(w1[o * in + k])", "oracle_bf16_to_double(w1[k * hid + o])"),
+    "bf16_half_ulp": ("uint32_t u = (uint32_t)b << 16;", "uint32_t u = ((uint32_t)b << 16) | 0x8000u;"),
+    # D-dimensional inputs (strings that occur only in the N-d functions)
+    "nd_weight_axis_swap": ("int64_t *vc)\n{\n    double w = 1.0;\n    for (int i = 0; i < D; ++i) {\n        int d = (c >> i) & 1;\n"
+                            "        vc[i] = v[i] + d;\n        w *= d ? frac[i] : 1.0 - frac[i];",
+                            "int64_t *vc)\n{\n    double w = 1.0;\n    for (int i = 0; i < D; ++i) {\n        int d = (c >> i) & 1;\n"
+                            "        vc[i] = v[i] + d;\n        w *= d ? frac[D - 1 - i] : 1.0 - frac[D - 1 - i];"),
+    "nd_scale_by_N_minus_1": ("double *frac)\n{\n    for (int i = 0; i < D; ++i) {\n        float xs = xp[i] * (float)res_l;",
+                              "double *frac)\n{\n    for (int i = 0; i < D; ++i) {\n        float xs = xp[i] * (float)(res_l - 1);"),
 }
 
 def _pin_calls():
