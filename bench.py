@@ -90,10 +90,9 @@ def csrc_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str, workload: str) -> float | None:
-    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of ``kernel`` on
-    ``workload`` from the committed ncu summary, or None when the kernel sources changed
-    since that capture."""
+def ncu_entry(kernel: str, workload: str) -> dict | None:
+    """The committed ncu figures of ``kernel`` on ``workload`` (profiles/ncu_traffic.json),
+    or None when the kernel sources changed since that capture."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -102,7 +101,12 @@ def ncu_traffic(kernel: str, workload: str) -> float | None:
         return None
     if d.get("csrc_sha") != csrc_digest():
         return None
-    ent = d.get("kernels", {}).get(f"{kernel}@{workload}")
+    return d.get("kernels", {}).get(f"{kernel}@{workload}")
+
+
+def ncu_traffic(kernel: str, workload: str) -> float | None:
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum), or None."""
+    ent = ncu_entry(kernel, workload)
     return None if ent is None else float(ent["dram_bytes_per_launch"])
 
 
@@ -472,10 +476,16 @@ def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, ke
     bytes_per_launch = algorithmic_bytes_per_point(w, kind) * points
     achieved = bytes_per_launch / (kernel_ms * 1e-3) / 1e9
     traffic = ncu_traffic(kernel, w.name)
-    return {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": traffic,
-            "algorithmic_bytes_per_launch": bytes_per_launch, "kernel_ms": round(kernel_ms, 5),
-            "peak_source": f"hbm_gbs of {src} peaks"}
+    out = {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+           "frac": round(achieved / peak, 4), "traffic": traffic,
+           "algorithmic_bytes_per_launch": bytes_per_launch, "kernel_ms": round(kernel_ms, 5),
+           "peak_source": f"hbm_gbs of {src} peaks"}
+    ent = ncu_entry(kernel, w.name)
+    if ent is not None and ent.get("l2_red_requests_per_launch"):
+        # what actually limits the backward: L2 reduction requests (counted by ncu) per second
+        reds = float(ent["l2_red_requests_per_launch"])
+        out["l2_red"] = {"requests_per_launch": int(reds), "achieved_g_per_s": round(reds / (kernel_ms * 1e-3) / 1e9, 1)}
+    return out
 
 
 def cpu_baseline(w: workloads.Workload, sample: int, budget_s: float = 10.0) -> dict:
