@@ -2,10 +2,13 @@
 
 The pages print no worked numbers for the encoding, so each pin here is derived from a
 closed form, an invariant, an exact integer computation or a brute-force formulation that
-is written differently from the oracle (see the docstring of each test). Together they are
+is written differently from the oracle (see the docstring of each test); the configuration
+values they do print (level table, table size, primes) are fixtures under tests/golden/. Together they are
 chosen so that a dropped corner, a swapped axis, a wrong sign, a wrong prime, a wrong
 resolution rounding or a deduplicated gradient each fails at least one of them.
 """
+import json
+import os
 from fractions import Fraction
 
 import numpy as np
@@ -605,3 +608,42 @@ def test_nd_backward_adjoint_and_input_gradient(D):
         xm[:, i] -= h
         fd = np.sum(up.astype(np.float64) * (g.forward(xp, t) - g.forward(xm, t)), axis=1) / (2 * float(h))
         np.testing.assert_allclose(dx[:, i], fd, rtol=1e-9, atol=1e-9)
+
+# ---------------------------------------------------------------------------------------
+# Values the pages print (tests/golden/, each file citing its page and section)
+# ---------------------------------------------------------------------------------------
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def test_golden_level_table():
+    t = golden("repro_hg_level_table.json")
+    r = oracle.resolutions(t["levels"], t["coarsest_resolution"], t["finest_resolution"])
+    assert r[0] == t["coarsest_resolution"] and r[-1] == t["finest_resolution"]
+    g = Grid(t["levels"], t["features"], t["log2_table_size"], t["coarsest_resolution"], t["finest_resolution"])
+    assert g.T == 2 ** 19 and g.L * g.F == 32
+    # the printed level-2 row is the table's inconsistency: the schedule gives 20 there
+    assert r[1] == 20 != t["printed_level_2_resolution"] and r[3] == t["printed_level_2_resolution"]
+
+
+def test_golden_parameter_count():
+    t = golden("nerface_hg_parameter_count.json")
+    g = Grid(t["levels"], t["features"], 19, 16, 512)
+    assert g.T == t["entries_per_level"]
+    assert g.L * g.T * g.F == 16 * 524288 * 2 == 16777216
+
+
+def test_golden_primes():
+    t = golden("hash_primes.json")
+    p3 = t["primes_3d"]
+    assert [oracle.hash3(1, 0, 0), oracle.hash3(0, 1, 0), oracle.hash3(0, 0, 1)] == p3
+    assert tuple(p3) == PRIMES
+    for i, prime in enumerate(t["primes_nd"]):
+        e = [0] * len(t["primes_nd"])
+        e[i] = 1
+        assert oracle.hash_nd(e) == prime
