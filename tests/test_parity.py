@@ -753,3 +753,20 @@ def test_cuda_graph_capture_and_replay():
     torch.cuda.synchronize()
     check_forward(og, inp2.x, inp.table, out.cpu().numpy(), "f32")
     assert rel_l2(d.cpu().numpy(), og.backward(inp2.x, inp2.g, nthreads=THREADS)) <= BWD_REL_L2
+
+
+# ---------------------------------------------------------------------------------------
+# The README's usage example runs as written
+# ---------------------------------------------------------------------------------------
+
+def test_readme_usage_example():
+    import os
+    import re
+    readme = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "README.md")
+    block = re.search(r"```python\n(.*?)```", open(readme).read(), re.S).group(1)
+    scope = {}
+    exec(compile(block, "README.md", "exec"), scope)
+    torch.cuda.synchronize()
+    assert scope["out"].shape == (1 << 20, 32) and torch.isfinite(scope["out"]).all()
+    assert scope["dL_dx"].shape == (1 << 20, 3) and torch.isfinite(scope["y"]).all()
+    assert int(torch.count_nonzero(scope["dL_dtable"])) == 0      # the Adam step cleared it
