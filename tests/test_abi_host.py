@@ -17,7 +17,9 @@ import multiresolution_hash_grid_b200 as hg
 from tests.test_oracle_pins import exact_floor_resolution, near_integer_from_below
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "hashgrid.h")
+INCLUDE_DIR = os.path.join(ROOT, "include")
+HEADER = os.path.join(INCLUDE_DIR, "hashgrid.h")
+LIB_PATH = os.path.join(ROOT, "multiresolution_hash_grid_b200", "libhashgrid.so")
 
 
 def declared_functions():
@@ -198,3 +200,42 @@ def test_binding_fails_loudly_without_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import multiresolution_hash_grid_b200"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "ImportError" in r.stderr and "not built" in r.stderr
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include "hashgrid.h"
+
+int main(void)
+{
+    hashgrid_t h = NULL;
+    int res[16], L, F, log2T, nmin, nmax, dtype;
+    if (hashgrid_create(16, 2, 19, 16, 512, HASHGRID_F32, &h) != HASHGRID_OK) {
+        fprintf(stderr, "%s\n", hashgrid_last_error());
+        return 1;
+    }
+    if (hashgrid_resolutions(h, res) != HASHGRID_OK || res[0] != 16 || res[15] != 512) return 2;
+    if (hashgrid_params(h, &L, &F, &log2T, &nmin, &nmax, &dtype) != HASHGRID_OK || L != 16 || F != 2) return 3;
+    if (hashgrid_table_elems(h) != (size_t)16 * 524288 * 2 || hashgrid_output_width(h) != 32) return 4;
+    /* an invalid call is an error code before any launch, with a message */
+    if (hashgrid_forward(h, NULL, 4, NULL, NULL, NULL) == HASHGRID_OK || hashgrid_last_error()[0] == 0) return 5;
+    hashgrid_destroy(h);
+    printf("%s\n", hashgrid_version());
+    return 0;
+}
+"""
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc missing")
+def test_header_is_plain_c_and_links(tmp_path):
+    """A C99 client compiled with gcc -Wall -Werror against include/hashgrid.h links to the
+    library and uses it without a GPU (create, queries, an argument error, destroy)."""
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", INCLUDE_DIR, str(src), "-o", str(exe),
+                    "-L", libdir, "-lhashgrid", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert "sm_100a" in r.stdout
