@@ -517,7 +517,10 @@ def check_mlp(og, x, table, wts, got):
 
 
 @pytest.mark.parametrize("shape", [(16, 2, 19, 16, 512, "f32"), (8, 2, 12, 4, 128, "f32"), (24, 2, 12, 4, 600, "f32"),
-                                   (16, 4, 14, 16, 4096, "f32"), (16, 2, 19, 16, 512, "f16")])
+                                   (16, 4, 14, 16, 4096, "f32"), (16, 2, 19, 16, 512, "f16"),
+                                   (16, 1, 12, 16, 512, "f32"), (32, 1, 10, 8, 1000, "f16"),     # F = 1: two levels per store
+                                   (4, 8, 12, 4, 200, "f32"), (8, 8, 12, 4, 300, "f16"),         # F = 8: 512-thread CTAs
+                                   (12, 4, 12, 4, 300, "f16")])
 def test_mlp_forward_parity(shape):
     hg = hgmod()
     L, F, log2T, a, b, dtype = shape
