@@ -709,6 +709,34 @@ def test_nd_parity(D, F):
     assert np.all(np.abs(dx - dxref) <= 1e-5 * B[:, None] * 2 ** (D - 3) + 1e-30)
 
 
+@pytest.mark.parametrize("F", [2, 4])
+@pytest.mark.parametrize("D", [2, 4])
+def test_nd_parity_fp16_table(D, F):
+    """fp16 tables with D = 2 and 4: the entries are decoded exactly, so the forward holds
+    the fp32 bound (1e-6 of sum_c w_c |e_c|) and dL/dx the same bound as with fp32 tables."""
+    hg = hgmod()
+    L, log2T = 6, 12
+    grid = hg.HashGrid(L, F, log2T, 3, 150, dtype=hg.HASHGRID_F16, D=D)
+    og = oracle.GridND(D, L, F, log2T, 3, 150, dtype=oracle.F16)
+    rng = np.random.default_rng(120 + 10 * D + F)
+    table = (rng.standard_normal((L, 2**log2T, F)) * 0.5).astype(np.float16)
+    x = rng.random((1500 + 11, D), dtype=np.float32)
+    g = workloads.upstream_grads(rng, x.shape[0], L * F)
+    x_d, t_d, g_d = dev(x), dev(table), dev(g)
+    out = grid.forward(x_d, t_d).cpu().numpy().astype(np.float64)
+    ref = og.forward(x, table, nthreads=THREADS)
+    bound = og.forward(x, np.abs(table), nthreads=THREADS)
+    assert np.all(np.abs(out - ref) <= 1e-6 * bound + 1e-30)
+    assert rel_l2(grid.backward(x_d, g_d).cpu().numpy(), og.backward(x, g, nthreads=THREADS)) <= BWD_REL_L2
+    dx = grid.backward_input(x_d, g_d, t_d).cpu().numpy().astype(np.float64)
+    dxref = og.backward_x(x, table, g, nthreads=THREADS)
+    tmax = float(np.max(np.abs(table.astype(np.float64))))
+    B = np.zeros(x.shape[0])
+    for l, n in enumerate(og.res):
+        B += float(n) * 2.0 * np.sum(np.abs(g[:, l * F:(l + 1) * F].astype(np.float64)), axis=1) * tmax
+    assert np.all(np.abs(dx - dxref) <= 1e-5 * B[:, None] * 2 ** (D - 3) + 1e-30)
+
+
 def test_nd_mlp_rejected():
     hg = hgmod()
     grid = hg.HashGrid(16, 2, 12, 16, 512, D=2)
