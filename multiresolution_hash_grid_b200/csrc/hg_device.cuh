@@ -1193,16 +1193,18 @@ __device__ __forceinline__ float adam_one(float& m, float& v, float theta, float
     return theta - a.lr * __fdiv_rn(m * a.c1, denom);
 }
 
+// One 4-element group: the state is loaded first, the update and stores come later, so a
+// thread can have two groups' loads in flight at once.
 template <typename TT>
-__global__ void __launch_bounds__(256) adam_kernel(TT* __restrict__ param, float* __restrict__ mom1,
-                                                   float* __restrict__ mom2, float* __restrict__ grad,
-                                                   int64_t n4, AdamParams a, int zero_grad) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
-        const float4 g = __ldcs(reinterpret_cast<const float4*>(grad) + i);
-        if (g.x == 0.f && g.y == 0.f && g.z == 0.f && g.w == 0.f) continue;
-        float4 m = reinterpret_cast<float4*>(mom1)[i];
-        float4 v = reinterpret_cast<float4*>(mom2)[i];
-        float th[4];
+struct AdamGroup {
+    float m[4], v[4], th[4];
+
+    __device__ __forceinline__ void load(const TT* __restrict__ param, const float* __restrict__ mom1,
+                                         const float* __restrict__ mom2, int64_t i) {
+        const float4 mm = reinterpret_cast<const float4*>(mom1)[i];
+        const float4 vv = reinterpret_cast<const float4*>(mom2)[i];
+        m[0] = mm.x; m[1] = mm.y; m[2] = mm.z; m[3] = mm.w;
+        v[0] = vv.x; v[1] = vv.y; v[2] = vv.z; v[3] = vv.w;
         if constexpr (sizeof(TT) == 4) {
             const float4 t = reinterpret_cast<const float4*>(param)[i];
             th[0] = t.x; th[1] = t.y; th[2] = t.z; th[3] = t.w;
@@ -1211,13 +1213,17 @@ __global__ void __launch_bounds__(256) adam_kernel(TT* __restrict__ param, float
             const float2 lo = h2_bits_to_f2(t.x), hi = h2_bits_to_f2(t.y);
             th[0] = lo.x; th[1] = lo.y; th[2] = hi.x; th[3] = hi.y;
         }
+    }
+
+    __device__ __forceinline__ void update_store(TT* __restrict__ param, float* __restrict__ mom1,
+                                                 float* __restrict__ mom2, float* __restrict__ grad, int64_t i,
+                                                 const float4& g, const AdamParams& a, int zero_grad) {
         const float gv[4] = {g.x, g.y, g.z, g.w};
-        float mv[4] = {m.x, m.y, m.z, m.w}, vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            if (gv[k] != 0.f) th[k] = adam_one(mv[k], vv[k], th[k], gv[k], a);
-        reinterpret_cast<float4*>(mom1)[i] = make_float4(mv[0], mv[1], mv[2], mv[3]);
-        reinterpret_cast<float4*>(mom2)[i] = make_float4(vv[0], vv[1], vv[2], vv[3]);
+            if (gv[k] != 0.f) th[k] = adam_one(m[k], v[k], th[k], gv[k], a);
+        reinterpret_cast<float4*>(mom1)[i] = make_float4(m[0], m[1], m[2], m[3]);
+        reinterpret_cast<float4*>(mom2)[i] = make_float4(v[0], v[1], v[2], v[3]);
         if constexpr (sizeof(TT) == 4) {
             reinterpret_cast<float4*>(param)[i] = make_float4(th[0], th[1], th[2], th[3]);
         } else {
@@ -1228,6 +1234,31 @@ __global__ void __launch_bounds__(256) adam_kernel(TT* __restrict__ param, float
             reinterpret_cast<uint2*>(param)[i] = t;
         }
         if (zero_grad) __stcs(reinterpret_cast<float4*>(grad) + i, make_float4(0.f, 0.f, 0.f, 0.f));
+    }
+};
+
+__device__ __forceinline__ bool any_nonzero(const float4& g) {
+    return g.x != 0.f || g.y != 0.f || g.z != 0.f || g.w != 0.f;
+}
+
+// Grid-stride over 4-element groups, two independent groups (i and i + stride) per step:
+// both gradient loads first, then the state of the groups with a nonzero gradient, then
+// the updates (measured latency-bound with one group per step).
+template <typename TT>
+__global__ void __launch_bounds__(256) adam_kernel(TT* __restrict__ param, float* __restrict__ mom1,
+                                                   float* __restrict__ mom2, float* __restrict__ grad,
+                                                   int64_t n4, AdamParams a, int zero_grad) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += 2 * stride) {
+        const int64_t j = i + stride;
+        const float4 g0 = __ldcs(reinterpret_cast<const float4*>(grad) + i);
+        const float4 g1 = j < n4 ? __ldcs(reinterpret_cast<const float4*>(grad) + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const bool u0 = any_nonzero(g0), u1 = any_nonzero(g1);
+        AdamGroup<TT> s0, s1;
+        if (u0) s0.load(param, mom1, mom2, i);
+        if (u1) s1.load(param, mom1, mom2, j);
+        if (u0) s0.update_store(param, mom1, mom2, grad, i, g0, a, zero_grad);
+        if (u1) s1.update_store(param, mom1, mom2, grad, j, g1, a, zero_grad);
     }
 }
 
