@@ -40,11 +40,17 @@ MUTATIONS = {
     "mlp_bias_dropped": ("            double s = (double)b2[o];", "            double s = 0.0;"),
     "mlp_w1_transposed": ("oracle_bf16_to_double(w1[o * in + k])", "oracle_bf16_to_double(w1[k * hid + o])"),
     "bf16_half_ulp": ("uint32_t u = (uint32_t)b << 16;", "uint32_t u = ((uint32_t)b << 16) | 0x8000u;"),
+    "mlp_second_relu_dropped": ("            a2[o] = s > 0.0 ? s : 0.0;", "            a2[o] = s;"),
+    "mlp_w2_transposed": ("oracle_bf16_to_double(w2[o * hid + k])", "oracle_bf16_to_double(w2[k * hid + o])"),
+    "mlp_w3_row_shift": ("oracle_bf16_to_double(w3[o * hid + k])", "oracle_bf16_to_double(w3[((o + 1) % nout) * hid + k])"),
     # D-dimensional inputs (strings that occur only in the N-d functions)
     "nd_weight_axis_swap": ("int64_t *vc)\n{\n    double w = 1.0;\n    for (int i = 0; i < D; ++i) {\n        int d = (c >> i) & 1;\n"
                             "        vc[i] = v[i] + d;\n        w *= d ? frac[i] : 1.0 - frac[i];",
                             "int64_t *vc)\n{\n    double w = 1.0;\n    for (int i = 0; i < D; ++i) {\n        int d = (c >> i) & 1;\n"
                             "        vc[i] = v[i] + d;\n        w *= d ? frac[D - 1 - i] : 1.0 - frac[D - 1 - i];"),
+    # the index export laid out [point][corner][level] (a wrong stride; same size, in bounds)
+    "nd_index_stride": ("idx[((size_t)p * L + l) * nc + c] = oracle_hash_nd(D, vc) & mask;",
+                        "idx[((size_t)p * nc + c) * L + l] = oracle_hash_nd(D, vc) & mask;"),
     "nd_scale_by_N_minus_1": ("double *frac)\n{\n    for (int i = 0; i < D; ++i) {\n        float xs = xp[i] * (float)res_l;",
                               "double *frac)\n{\n    for (int i = 0; i < D; ++i) {\n        float xs = xp[i] * (float)(res_l - 1);"),
 }

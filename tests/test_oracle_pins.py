@@ -499,24 +499,95 @@ def test_bf16_decode():
         assert (got == want) or (np.isnan(got) and np.isnan(want))
 
 
-def test_mlp_matches_numpy_matmuls():
-    """The MLP of the oracle is three numpy matmuls with ReLU on the oracle's own fp64
-    encoding and the exactly decoded bf16 weights (a library routine for each layer)."""
-    g = Grid(16, 2, 12, 16, 512)
-    rng = np.random.default_rng(60)
-    table = (rng.standard_normal((16, 2**12, 2)) * 0.5).astype(np.float32)
-    x = rng.random((300, 3), dtype=np.float32)
-    w1 = bf16_bits(rng.standard_normal((64, 32)) * 0.3)
-    w2 = bf16_bits(rng.standard_normal((64, 64)) * 0.2)
-    w3 = bf16_bits(rng.standard_normal((4, 64)) * 0.2)
-    b1, b2, b3 = (rng.standard_normal(n).astype(np.float32) * 0.1 for n in (64, 64, 4))
-    y = g.mlp_forward(x, table, w1, b1, w2, b2, w3, b3)
-    e = g.forward(x, table)
-    a1 = np.maximum(e @ bf16_values(w1).T + b1.astype(np.float64), 0.0)
-    a2 = np.maximum(a1 @ bf16_values(w2).T + b2.astype(np.float64), 0.0)
-    want = a2 @ bf16_values(w3).T + b3.astype(np.float64)
-    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
-    assert np.any(a1 == 0) and np.any(a1 > 0)           # ReLU active on both sides
+# Pins of the MLP that the mathematics fixes exactly. The grid doubles its resolution at
+# every level (N 4 -> 2^17, b = 2), so x = k/4 is a vertex at every level and the encoding is
+# the table entry at the hashed vertex, exactly (P2); the entry is found here with Python big
+# ints, not with the oracle. Tables hold small integers and the weights are 0, +-1 or small
+# integers, all exact in bf16, so every layer is exact in fp64 and the pins compare exactly.
+MLP_GRID = (16, 2, 10, 4, 2**17)     # L, F, log2T, N_min, N_max: in = L*F = 32
+
+
+def mlp_vertex_inputs(seed):
+    L, F, log2T, nmin, nmax = MLP_GRID
+    rng = np.random.default_rng(seed)
+    table = rng.integers(-4, 5, size=(L, 2**log2T, F)).astype(np.float32)
+    k = np.stack(np.meshgrid(*[np.arange(5)] * 3, indexing="ij"), -1).reshape(-1, 3)
+    x = (k / 4.0).astype(np.float32)
+    e = np.zeros((len(k), L * F))
+    for p, kp in enumerate(k):
+        for l in range(L):
+            v = [int(ki) * (nmin << l) // 4 for ki in kp]          # x * N_l, an integer
+            e[p, l * F:(l + 1) * F] = table[l, bigint_hash(*v) % 2**log2T]
+    return Grid(*MLP_GRID), x, table, e
+
+
+def bf16_int(a):
+    """bf16 bit patterns of small integers (exact)."""
+    return bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def test_mlp_split_weights_give_absolute_values():
+    """W1 = [I; -I], b1 = 0 gives a1 = (relu(e), relu(-e)); W2 a permutation, b2 = 0 keeps
+    them; W3's first row of ones sums them: y0 = sum_k |e_k| + b3_0. Its second row weights
+    the permuted activations by 1..64, which fixes which activation each W2 row reads."""
+    g, x, table, e = mlp_vertex_inputs(61)
+    n = 32
+    w1 = np.zeros((64, n))
+    w1[:n, :n] = np.eye(n)
+    w1[n:, :n] = -np.eye(n)
+    perm = np.random.default_rng(62).permutation(64)
+    w2 = np.eye(64)[perm]                         # a2_j = a1_perm[j]
+    w3 = np.zeros((4, 64))
+    w3[0] = 1.0
+    w3[1] = np.arange(1, 65)
+    b1, b2 = np.zeros(64, np.float32), np.zeros(64, np.float32)
+    b3 = np.array([3.0, -5.0, 0.0, 7.0], np.float32)
+    y = g.mlp_forward(x, table, bf16_int(w1), b1, bf16_int(w2), b2, bf16_int(w3), b3)
+    np.testing.assert_array_equal(y[:, 0], np.abs(e).sum(1) + 3.0)
+    a1 = np.concatenate([np.maximum(e, 0), np.maximum(-e, 0)], 1)
+    np.testing.assert_array_equal(y[:, 1], (a1[:, perm] * np.arange(1, 65)).sum(1) - 5.0)
+    np.testing.assert_array_equal(y[:, 2], 0.0)
+    np.testing.assert_array_equal(y[:, 3], 7.0)
+    assert np.any(e < 0) and np.any(e > 0)
+
+
+def test_mlp_first_relu_zeroes_negative_preactivations():
+    """W1 = I, b1 = -1: a1_k = max(e_k - 1, 0), so every entry below 1 is cut to zero;
+    W2 = I, b2 = 100 keeps layer 2 linear (a2 = a1 + 100 > 0, so its own ReLU cannot redo
+    the cut); y0 = sum_k max(e_k - 1, 0) + 32 * 100."""
+    g, x, table, e = mlp_vertex_inputs(63)
+    w1 = np.zeros((64, 32))
+    w1[:32] = np.eye(32)
+    w3 = np.zeros((4, 64))
+    w3[0, :32] = 1.0
+    b1 = np.full(64, -1.0, np.float32)
+    b2 = np.full(64, 100.0, np.float32)
+    y = g.mlp_forward(x, table, bf16_int(w1), b1, bf16_int(np.eye(64)), b2, bf16_int(w3), np.zeros(4, np.float32))
+    np.testing.assert_array_equal(y[:, 0], np.maximum(e - 1.0, 0).sum(1) + 3200.0)
+    assert np.any(e < 1) and np.any(e > 1)
+
+
+def test_mlp_second_relu_zeroes_negative_preactivations():
+    """W1 = I, b1 = 100 keeps layer 1 linear (a1 = e + 100 > 0); W2 = -I, b2 = 101 gives
+    a2_k = max(1 - e_k, 0), cut to zero wherever e_k > 1; y0 = sum_k max(1 - e_k, 0), with
+    rows of W3 = 2 and a bias added to the other outputs."""
+    g, x, table, e = mlp_vertex_inputs(64)
+    w1 = np.zeros((64, 32))
+    w1[:32] = np.eye(32)
+    w3 = np.zeros((4, 64))
+    w3[0, :32] = 1.0
+    w3[2, :32] = 2.0
+    b1 = np.full(64, 100.0, np.float32)
+    b2 = np.full(64, 101.0, np.float32)
+    b2[32:] = -1.0                                # rows with no input: relu(-1) = 0
+    b3 = np.array([0.0, 1.5, 0.25, -2.0], np.float32)
+    y = g.mlp_forward(x, table, bf16_int(w1), b1, bf16_int(-np.eye(64)), b2, bf16_int(w3), b3)
+    want = np.maximum(1.0 - e, 0).sum(1)
+    np.testing.assert_array_equal(y[:, 0], want)
+    np.testing.assert_array_equal(y[:, 1], 1.5)
+    np.testing.assert_array_equal(y[:, 2], 2 * want + 0.25)
+    np.testing.assert_array_equal(y[:, 3], -2.0)
+    assert np.any(e > 1) and np.any(e < 1)
 
 
 # ---------------------------------------------------------------------------------------
@@ -544,6 +615,28 @@ def test_hash_nd_bigint_and_primes():
             e[i] = 1
             assert oracle.hash_nd(e) == PRIMES7[i]
     assert oracle.hash_nd([1, 1, 1, 1]) == 1 ^ 2654435761 ^ 805459861 ^ 3674653429
+
+
+@pytest.mark.parametrize("D", [2, 4])
+def test_nd_indices_equal_bigint_hash_of_every_corner(D):
+    """Every exported index of a D-dimensional point equals the big-int hash of
+    floor(fp32(x_i * N_l)) + offset_i mod T, corner c having offset bit i = (c >> i) & 1,
+    laid out [point][level][corner]; points inside, on and outside the unit cube."""
+    L, log2T = 5, 12
+    g = oracle.GridND(D, L, 2, log2T, 3, 300)
+    rng = np.random.default_rng(96 + D)
+    x = (rng.random((150, D)) * 2.0 - 0.5).astype(np.float32)
+    x[0] = 0.0
+    x[1] = 1.0
+    x[2] = np.float32(1.0 - 2**-24)
+    idx = g.indices(x)
+    assert idx.shape == (150, L, 2**D)
+    for p in range(150):
+        for l, n in enumerate(g.res):
+            v = [int(np.floor(np.float32(x[p, i]) * np.float32(n))) for i in range(D)]
+            for c in range(2**D):
+                corner = [v[i] + ((c >> i) & 1) for i in range(D)]
+                assert idx[p, l, c] == bigint_hash_nd(corner, 2**log2T), (p, l, c)
 
 
 def test_nd_at_three_dimensions_equals_3d_oracle():
