@@ -53,9 +53,9 @@ CPU_SAMPLE_POINTS = 1 << 18
 REFERENCE_SAMPLE_POINTS = 1 << 17
 NEXT_ROWS_CPU_SAMPLE = 1 << 16
 FALLBACK_HBM_GBS = 6650.0
-GATHER_MODES = {"auto": 0, "corner": 1, "sector": 2, "pair": 3}  # HASHGRID_GATHER_*
+GATHER_MODES = {"auto": 0, "corner": 1, "sector": 2, "pair": 3, "lanes": 4}  # HASHGRID_GATHER_*
 SCHEDULES = {"auto": 0, "point": 1, "level": 2}             # HASHGRID_SCHEDULE_*
-BACKWARD_MODES = {"auto": 0, "atomic": 1, "dedup": 2, "runs": 3, "dedup_adaptive": 4}  # HASHGRID_BACKWARD_*
+BACKWARD_MODES = {"auto": 0, "atomic": 1, "dedup": 2, "runs": 3, "dedup_adaptive": 4, "run_lanes": 5}  # HASHGRID_BACKWARD_*
 
 
 # ---------------------------------------------------------------------------------------
@@ -79,6 +79,66 @@ def measured_peaks() -> tuple[float, str]:
             return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------------------
+# Memory-system peaks of the gather / reduction roofline, measured in the same run
+# ---------------------------------------------------------------------------------------
+
+PEAK_BUFFERS = {"32MiB": 32 << 20, "64MiB": 64 << 20}   # both stay in L2 (126 MB)
+PEAK_OPS = 1 << 26               # lane operations per probe launch (~0.2-0.5 ms)
+PROBE_PATTERNS = {"random": 0, "xpair": 1, "sector_pair": 2, "line_pair": 3, "stream": 4}
+
+
+def probe_rate(kind: int, width: int, pattern: str, buf, sink, device, reps: int = 5) -> float:
+    """Median lane operations per second of one probe (include/hashgrid_probe.h) over
+    ``reps`` launches timed with CUDA events, after two untimed ones."""
+    import torch
+    import multiresolution_hash_grid_b200 as hg
+    stream = torch.cuda.current_stream(device)
+    nbytes = buf.numel() * buf.element_size()
+    for _ in range(2):
+        hg.hashgrid_probe(kind, width, PROBE_PATTERNS[pattern], buf, nbytes, PEAK_OPS, sink)
+    ts, done = [], 0
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        done = hg.hashgrid_probe(kind, width, PROBE_PATTERNS[pattern], buf, nbytes, PEAK_OPS, sink)
+        b.record(stream)
+        ts.append((a, b))
+    torch.cuda.synchronize(device)
+    return done / (statistics.median(x.elapsed_time(y) for x, y in ts) * 1e-3)
+
+
+def measure_l2_peaks(device) -> dict:
+    """Rates of the encoding's own accesses on buffers that stay in L2 (32 and 64 MiB, the
+    sizes of the fp16 and fp32 default tables and of one level of the 1 GiB grid), in lane
+    operations per second: gathers of 4 to 16 bytes (a table entry of F*s bytes) and fp32 /
+    fp16 reductions of 4 to 16 bytes (one corner's F-wide contribution), each with
+    independent random units and with the hash's x-neighbour pairs (two lanes of an
+    instruction on units v XOR K and (v + 1) XOR K: the access pattern of the lane-pair
+    kernels); plus 32-byte random gathers and a coalesced sweep for context."""
+    import torch
+    import multiresolution_hash_grid_b200 as hg
+    kinds = {"gather": hg.HASHGRID_PROBE_GATHER, "red": hg.HASHGRID_PROBE_RED, "red_f16": hg.HASHGRID_PROBE_RED_F16}
+    out = {"ops_per_launch": PEAK_OPS, "unit": "G lane operations/s",
+           "method": "hashgrid_probe kernels (8 blocks x 256 threads per SM, 8 independent operations in flight "
+                     "per thread), median of 5 launches timed with CUDA events after 2 untimed ones",
+           "buffers": {}}
+    sink = torch.zeros(1, dtype=torch.float32, device=device)
+    for key, nbytes in PEAK_BUFFERS.items():
+        buf = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        b = {}
+        for kname, kind in kinds.items():
+            b[kname] = {}
+            for w in (4, 8, 16):
+                b[kname][str(w)] = {pat: round(probe_rate(kind, w, pat, buf, sink, device) / 1e9, 2)
+                                    for pat in ("random", "xpair")}
+        b["gather"]["32"] = {"random": round(probe_rate(kinds["gather"], 32, "random", buf, sink, device) / 1e9, 2)}
+        b["stream_read_gbs"] = round(probe_rate(kinds["gather"], 16, "stream", buf, sink, device) * 16 / 1e9, 1)
+        out["buffers"][key] = b
+        del buf
+    return out
 
 
 def csrc_digest() -> str:
@@ -232,12 +292,12 @@ class Resident:
     """One workload's inputs and outputs resident in HBM, plus the library handle."""
 
     def __init__(self, w: workloads.Workload, seed: int, device, backward: bool,
-                 gather: str = "auto", backward_mode: str = "auto", schedule: str = "auto"):
+                 gather: str = "auto", backward_mode: str = "auto", schedule: str = "auto", points: int | None = None):
         import torch
 
         import multiresolution_hash_grid_b200 as hg
         self.w, self.hg, self.backward = w, hg, backward
-        inp = workloads.make_inputs(w, seed=seed, grads=backward)
+        inp = workloads.make_inputs(w, seed=seed, n_points=points, grads=backward)
         self.N = inp.x.shape[0]
         self.x = torch.from_numpy(inp.x).to(device)
         self.table = torch.from_numpy(inp.table).to(device)
@@ -261,10 +321,21 @@ class Resident:
         self.hg.hashgrid_destroy(self.handle)
 
 
-def time_steps(res: Resident, steps: int, warmup: int, device, sampler=None) -> dict:
-    """Times ``steps`` steps with CUDA events on the launching stream. Each step: forward,
-    zero the gradient and backward (if backward). L2 is flushed before every step, outside
-    the step's events. Returns per-phase mean milliseconds and the max-over-ranks total."""
+def loop_repeats(steps: int, step_s: float, min_timed_s: float) -> int:
+    """How many times the K-step loop runs back to back in the timed region so that the
+    region lasts at least ``min_timed_s`` (at least once)."""
+    if min_timed_s <= 0 or step_s <= 0:
+        return 1
+    return max(1, int(-(-min_timed_s // (steps * step_s))))
+
+
+def time_steps(res: Resident, steps: int, warmup: int, device, sampler=None, min_timed_s: float = 0.0) -> dict:
+    """Times steps with CUDA events on the launching stream. Each step: forward, zero the
+    gradient and backward (if backward). L2 is flushed before every step, outside the
+    step's events. The timed region runs the K-step loop R times back to back (R from the
+    warm-up's wall time so that the region lasts at least ``min_timed_s``; R is the same
+    on every rank), and every one of the R * K steps is timed. Returns per-phase mean
+    milliseconds, the max-over-ranks total and R."""
     import torch
     stream = torch.cuda.current_stream(device)
     sp = stream.cuda_stream
@@ -289,15 +360,21 @@ def time_steps(res: Resident, steps: int, warmup: int, device, sampler=None) -> 
         if evs:
             evs[3].record(stream)
 
+    torch.cuda.synchronize(device)
+    t0 = time.perf_counter()
     for _ in range(warmup):
         one()
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    torch.cuda.synchronize(device)
+    step_s = (time.perf_counter() - t0) / max(warmup, 1)
+    repeats = int(max_over_ranks(float(loop_repeats(steps, step_s, min_timed_s)), device))
+    n = steps * repeats
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
     torch.cuda.synchronize(device)
     barrier(device)
     torch.cuda.synchronize(device)
     if sampler is not None:
         sampler.__enter__()
-    for k in range(steps):
+    for k in range(n):
         one(events[k])
     torch.cuda.synchronize(device)
     if sampler is not None:
@@ -306,7 +383,7 @@ def time_steps(res: Resident, steps: int, warmup: int, device, sampler=None) -> 
     torch.cuda.synchronize(device)
     fwd = [e[0].elapsed_time(e[1]) for e in events]
     zero = [e[1].elapsed_time(e[2]) for e in events]
-    bwd = [e[2].elapsed_time(e[3]) for e in events] if res.backward else [0.0] * steps
+    bwd = [e[2].elapsed_time(e[3]) for e in events] if res.backward else [0.0] * n
     total = [e[0].elapsed_time(e[3]) for e in events]
     total_ms = sum(total)
     return {
@@ -314,7 +391,8 @@ def time_steps(res: Resident, steps: int, warmup: int, device, sampler=None) -> 
         "max_total_ms": max_over_ranks(total_ms, device),
         "zero_ms": statistics.mean(zero), "fwd_ms": statistics.mean(fwd), "bwd_ms": statistics.mean(bwd),
         "step_ms": statistics.mean(total),
-        "launches": steps * (2 if res.backward else 1),
+        "repeats": repeats, "timed_steps": n,
+        "launches": n * (2 if res.backward else 1),
     }
 
 
@@ -402,7 +480,7 @@ def time_launches(fn, steps: int, warmup: int, device, before=None) -> float:
     return statistics.mean(a.elapsed_time(b) for a, b in ts)
 
 
-def time_next_rows(res: Resident, steps: int, warmup: int, device) -> tuple[dict, int]:
+def time_next_rows(res: Resident, steps: int, warmup: int, device, l2peaks=None) -> tuple[dict, int]:
     """The operations beyond the forward/backward pair, on the same resident batch: the
     gradient w.r.t. x, one sparse Adam step over the table, the encoding fused with the
     3-layer MLP on the tensor cores, and the backward into an fp16 gradient table. Each is
@@ -466,25 +544,77 @@ def time_next_rows(res: Resident, steps: int, warmup: int, device) -> tuple[dict
     dh = torch.zeros((w.L, w.T, w.F), dtype=torch.float16, device=device)
     ms = time_launches(lambda: hg.hashgrid_backward_half(res.handle, res.x, res.g, N, dh, sp), steps, warmup,
                        device, before=dh.zero_)
-    out["backward_half"] = entry(ms, N * (12 + 4 * LF + 8 * LF * 2), "backward_kernel_half")
+    out["backward_half"] = {"ms": round(ms, 5), "points_per_s": round(N / (ms * 1e-3), 1),
+                            "roofline": roofline(w, "bwd", N, ms, "backward_kernel_half", l2peaks, grad_dtype="f16")}
     launches += steps
     return out, launches
 
 
-def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, kernel: str) -> dict:
-    peak, src = measured_peaks()
-    bytes_per_launch = algorithmic_bytes_per_point(w, kind) * points
-    achieved = bytes_per_launch / (kernel_ms * 1e-3) / 1e9
-    traffic = ncu_traffic(kernel, w.name)
-    out = {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-           "frac": round(achieved / peak, 4), "traffic": traffic,
-           "algorithmic_bytes_per_launch": bytes_per_launch, "kernel_ms": round(kernel_ms, 5),
+L2_RESIDENT_BYTES = 96 << 20   # a kernel's table (or gradient) working set that stays in L2
+
+
+def stream_bytes_per_point(w: workloads.Workload, kind: str) -> int:
+    """HBM-compulsory bytes of one point: x in, and the output (fwd) or the upstream
+    gradient (bwd) rows."""
+    return 12 + 4 * w.L * w.F
+
+
+def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, kernel: str,
+             l2peaks: dict | None, grad_dtype: str = "f32") -> dict:
+    """Roofline of one kernel launch over ``points`` points (kind "fwd" or "bwd").
+
+    HBM (the primary fraction, bound "hbm"): the algorithmic bytes of the launch (x, the
+    table gathers or fp32 reductions counted once each, the output or upstream-gradient
+    rows) at the measured HBM copy bandwidth.
+    L2 (the benchmark spec: the gather roofline is L2 for tables that fit in it): the 8 * L table
+    gathers (fwd) or corner reductions (bwd) per point at the rate this device serves the
+    hash's access pattern from an L2-resident buffer of the working set's size: x-neighbour
+    pairs of F*s-byte entries (fwd) or F-wide fp32 / fp16 contributions (bwd), measured in
+    the same run by the probe kernels. The working set is the table (fwd) or gradient
+    (bwd), or one level of it under the level-major schedule (tables above 96 MB).
+    bound_time is the larger of the L2 time and the time of the bytes that must cross HBM
+    (all of them for a table larger than L2, else the x / output / upstream-gradient
+    rows); frac_bound_time = bound_time / kernel time. Batches more coherent than the
+    probe's independent random pairs (samples along rays share cache lines and voxels)
+    can exceed 1 on the L2 basis."""
+    hbm, src = measured_peaks()
+    s = 2 if w.dtype == "f16" else 4
+    alg = algorithmic_bytes_per_point(w, kind) * points
+    if kind == "bwd" and grad_dtype == "f16":
+        alg = (12 + 4 * w.L * w.F + 8 * w.L * w.F * 2) * points
+    hbm_gbs = alg / (kernel_ms * 1e-3) / 1e9
+    elem = s if kind == "fwd" else (2 if grad_dtype == "f16" else 4)
+    table_bytes = w.L * w.T * w.F * elem
+    level_major = w.L * w.T * w.F * s > L2_RESIDENT_BYTES
+    working_set = table_bytes // w.L if level_major else table_bytes
+    in_l2 = working_set <= L2_RESIDENT_BYTES
+    out = {"bound": "hbm", "kernel": kernel, "kernel_ms": round(kernel_ms, 5), "unit": "GB/s",
+           "achieved": round(hbm_gbs, 1), "peak": hbm, "frac": round(hbm_gbs / hbm, 4),
+           "traffic": ncu_traffic(kernel, w.name), "algorithmic_bytes_per_launch": alg,
            "peak_source": f"hbm_gbs of {src} peaks"}
+    t_stream = (alg if not (in_l2 and not level_major) else stream_bytes_per_point(w, kind) * points) / (hbm * 1e9)
+    t_l2 = 0.0
+    if l2peaks is not None and in_l2:
+        ops = 8 * w.L * points
+        width = w.F * elem
+        bkey = "32MiB" if working_set <= (32 << 20) else "64MiB"
+        pk = "gather" if kind == "fwd" else ("red_f16" if grad_dtype == "f16" else "red")
+        rates = l2peaks["buffers"][bkey][pk][str(width)]
+        t_l2 = ops / (rates["xpair"] * 1e9)
+        out["l2"] = {"access": (f"{width}-byte table gathers" if kind == "fwd" else
+                                f"{width}-byte {grad_dtype} corner reductions") + ", 8 per point and level",
+                     "ops_per_launch": ops, "achieved_g_ops_per_s": round(ops / (kernel_ms * 1e-3) / 1e9, 1),
+                     "peak_g_ops_per_s": rates["xpair"], "frac": round(t_l2 / (kernel_ms * 1e-3), 4),
+                     "frac_vs_random_units": round(ops / (rates["random"] * 1e9) / (kernel_ms * 1e-3), 4),
+                     "peak_source": f"hashgrid_probe, x-neighbour pairs on a {bkey} L2-resident buffer, this run"}
+    bound_s = max(t_stream, t_l2)
+    out["bound_time_ms"] = round(bound_s * 1e3, 5)
+    out["bound_by"] = "l2" if t_l2 >= t_stream else "hbm"
+    out["frac_bound_time"] = round(bound_s / (kernel_ms * 1e-3), 4)
     ent = ncu_entry(kernel, w.name)
     if ent is not None and ent.get("l2_red_requests_per_launch"):
-        # what actually limits the backward: L2 reduction requests (counted by ncu) per second
         reds = float(ent["l2_red_requests_per_launch"])
-        out["l2_red"] = {"requests_per_launch": int(reds), "achieved_g_per_s": round(reds / (kernel_ms * 1e-3) / 1e9, 1)}
+        out["l2_red_requests"] = {"per_launch": int(reds), "g_per_s": round(reds / (kernel_ms * 1e-3) / 1e9, 1)}
     return out
 
 
@@ -609,6 +739,40 @@ def run_reference(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+LEGS = ("grid_L16F2T19", "half_L16F2T19", "large_L16F4T22")   # timed besides the step's workload
+
+
+def time_workload(w: workloads.Workload, args, device, rank: int, world: int, l2peaks, min_timed_s: float,
+                  sampler=None) -> tuple[dict, Resident, int]:
+    """Times one workload's step (forward, or forward + zero + backward) and returns its
+    JSON object (rate, phases, a roofline per kernel), the resident inputs and the number
+    of timed launches."""
+    res = Resident(w, rank_seed(rank), device, backward=w.backward, gather=args.forward_gather,
+                   backward_mode=args.backward_mode, schedule=args.schedule,
+                   points=args.points if w.name == args.workload else None)
+    t = time_steps(res, args.steps, args.warmup, device, sampler, min_timed_s=min_timed_s)
+    n = t["timed_steps"]
+    seconds = t["max_total_ms"] * 1e-3
+    obj = {"workload": w.name, "description": w.describe(), "value": round(whole_job_rate(res.N * n, world, seconds), 1),
+           "unit": UNIT, "ms_per_step": round(t["max_total_ms"] / n, 5), "points_per_rank": res.N,
+           "timed_steps": n, "loop_repeats": t["repeats"],
+           "phase_ms": {"fwd": round(t["fwd_ms"], 5), "zero": round(t["zero_ms"], 5), "bwd": round(t["bwd_ms"], 5)},
+           "rooflines": {"fwd": roofline(w, "fwd", res.N, t["fwd_ms"], "forward_kernel", l2peaks)}}
+    if w.backward:
+        obj["rooflines"]["bwd"] = roofline(w, "bwd", res.N, t["bwd_ms"], "backward_kernel", l2peaks)
+        hbm, src = measured_peaks()
+        step_bytes = algorithmic_bytes_per_point(w, "fwdbwd") * res.N
+        step_gbs = step_bytes / (t["step_ms"] * 1e-3) / 1e9
+        bound_ms = obj["rooflines"]["fwd"]["bound_time_ms"] + obj["rooflines"]["bwd"]["bound_time_ms"]
+        obj["roofline_step"] = {"achieved": round(step_gbs, 1), "peak": hbm, "unit": "GB/s",
+                                "frac": round(step_gbs / hbm, 4),
+                                "bound_time_ms": round(bound_ms, 5),
+                                "frac_bound_time": round(bound_ms / t["step_ms"], 4),
+                                "note": f"whole step incl. gradient zeroing; frac against the {src} HBM peak, "
+                                        "frac_bound_time = (fwd + bwd bound times) / step time"}
+    return obj, res, t["launches"]
+
+
 def run_b200(args) -> None:
     import torch
     rank, world, local = dist_env()
@@ -619,21 +783,16 @@ def run_b200(args) -> None:
     device = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(device)
     w = workloads.WORKLOADS[args.workload]
+    l2peaks = None if args.skip_peaks else measure_l2_peaks(device)
 
-    res = Resident(w, rank_seed(rank), device, backward=w.backward, gather=args.forward_gather,
-                   backward_mode=args.backward_mode, schedule=args.schedule)
     sampler = ClockSampler(device.index)
-    t = time_steps(res, args.steps, args.warmup, device, sampler)
-    seconds = t["max_total_ms"] * 1e-3
-    value = whole_job_rate(res.N * args.steps, world, seconds)
-    launches = t["launches"]
-
-    kind, kms, kname = ("bwd", t["bwd_ms"], "backward_kernel") if t["bwd_ms"] >= t["fwd_ms"] else \
-        ("fwd", t["fwd_ms"], "forward_kernel")
+    main, res, launches = time_workload(w, args, device, rank, world, l2peaks, args.min_timed_s, sampler)
+    rl = main["rooflines"]
+    kind = "bwd" if w.backward and main["phase_ms"]["bwd"] >= main["phase_ms"]["fwd"] else "fwd"
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(t["max_total_ms"] / args.steps, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "metric": METRIC, "value": main["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": main["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16" if w.dtype == "f16" else "f32",
         "data": "synthetic (seeded NeRF-like ray samples; random table)",
         "config": {"workload": w.name, "description": w.describe(), "points_per_rank": res.N,
                    "global_points": res.N * world, "parallelism": f"dp{world}: points sharded, no collective",
@@ -641,34 +800,35 @@ def run_b200(args) -> None:
                    "modes": {"forward_gather": args.forward_gather, "backward": args.backward_mode,
                              "schedule": args.schedule},
                    "l2": "flushed before every timed step (256 MiB write, outside the events)",
-                   "phase_ms": {"zero": round(t["zero_ms"], 5), "fwd": round(t["fwd_ms"], 5),
-                                "bwd": round(t["bwd_ms"], 5)}},
-        "roofline": roofline(w, kind, res.N, kms, kname),
-        "roofline_step": None,
+                   "timed_region": f"the {args.steps}-step loop run {main['loop_repeats']} times back to back "
+                                   f"({main['timed_steps']} steps, all timed) so that it lasts >= {args.min_timed_s} s",
+                   "phase_ms": main["phase_ms"]},
+        "roofline": rl[kind],
+        "roofline_step": main.get("roofline_step"),
+        "rooflines": rl,
         "clocks": sampler.summary(),
     }
-    step_bytes = algorithmic_bytes_per_point(w, "fwdbwd" if w.backward else "fwd") * res.N
-    peak, src = measured_peaks()
-    step_gbs = step_bytes / (t["step_ms"] * 1e-3) / 1e9
-    line["roofline_step"] = {"achieved": round(step_gbs, 1), "peak": peak, "unit": "GB/s",
-                             "frac": round(step_gbs / peak, 4),
-                             "note": f"whole step incl. gradient zeroing, {src} peak"}
+    if l2peaks is not None:
+        line["peaks"] = {"l2": l2peaks}
 
-    if not args.skip_fwd_leg and w.name != FWD_WORKLOAD:
-        fw = workloads.WORKLOADS[FWD_WORKLOAD]
-        fres = Resident(fw, rank_seed(rank), device, backward=False, gather=args.forward_gather,
-                        schedule=args.schedule)
-        ft = time_steps(fres, args.steps, args.warmup, device)
-        fval = whole_job_rate(fres.N * args.steps, world, ft["max_total_ms"] * 1e-3)
-        line["fwd"] = {"workload": fw.name, "description": fw.describe(), "value": round(fval, 1), "unit": UNIT,
-                       "ms_per_step": round(ft["max_total_ms"] / args.steps, 5),
-                       "roofline": roofline(fw, "fwd", fres.N, ft["fwd_ms"], "forward_kernel")}
-        launches += ft["launches"]
-        fres.close()
-        del fres
+    if not args.skip_legs:
+        legs = {}
+        for name in LEGS:
+            if name == w.name:
+                continue
+            lw = workloads.WORKLOADS[name]
+            obj, lres, n = time_workload(lw, args, device, rank, world, l2peaks, 0.0)
+            lres.close()
+            del lres
+            torch.cuda.empty_cache()
+            legs[name] = obj
+            launches += n
+        line["legs"] = legs
+        if "grid_L16F2T19" in legs:          # the metric's forward-only figure
+            line["fwd"] = legs["grid_L16F2T19"]
 
     if not args.skip_next_rows and w.backward:
-        line["next_rows"], n = time_next_rows(res, min(args.steps, 20), min(args.warmup, 3), device)
+        line["next_rows"], n = time_next_rows(res, min(args.steps, 20), min(args.warmup, 3), device, l2peaks)
         launches += n
         if rank == 0 and world == 1 and not args.skip_cpu_baseline:
             line["next_rows"]["cpu_oracle"] = cpu_next_rows(w, min(NEXT_ROWS_CPU_SAMPLE, res.N))
@@ -692,7 +852,50 @@ def run_b200(args) -> None:
         dist.destroy_process_group()
 
 
+def free_port() -> int:
+    import socket
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    port = sk.getsockname()[1]
+    sk.close()
+    return port
+
+
+def spawn_ranks(gpus: int, argv: list[str]) -> int:
+    """``--gpus N`` (N > 1) without a launcher: start N ranks of this script on this node
+    with torch.distributed.run (one process per GPU, rendezvous on 127.0.0.1) and return
+    its exit status. The ranks find WORLD_SIZE set and do not spawn again."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.abspath(__file__), *argv]
+    return subprocess.run(cmd).returncode
+
+
+def run_stub(args) -> None:
+    """The rank plumbing without a GPU (gloo, CPU): each rank sleeps a fixed time per step
+    in place of the GPU step, and rank 0 prints a line marked ``"impl": "stub"`` with the
+    world size, the max-over-ranks time and the whole-job rate. Tests use it to check that
+    ``--gpus N`` starts N ranks and that they agree on one line."""
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1:
+        dist.init_process_group("gloo", timeout=timedelta(seconds=60))
+    units = 1 << 20
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time.sleep(0.002 * (1 + rank))
+    dt = max_over_ranks(time.perf_counter() - t0)
+    barrier()
+    if rank == 0:
+        print(json.dumps({"impl": "stub", "metric": METRIC, "value": round(whole_job_rate(units * args.steps, world, dt), 1),
+                          "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": round(dt / args.steps * 1e3, 3), "scaling": "weak"}), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main(argv=None) -> None:
+    argv = list(sys.argv[1:] if argv is None else argv)
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -704,16 +907,29 @@ def main(argv=None) -> None:
     ap.add_argument("--schedule", choices=sorted(SCHEDULES), default="auto")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
-    ap.add_argument("--skip-fwd-leg", action="store_true")
+    ap.add_argument("--skip-legs", "--skip-fwd-leg", dest="skip_legs", action="store_true",
+                    help="skip timing the other workloads (forward-only grid, fp16 table, 1 GiB grid)")
+    ap.add_argument("--skip-peaks", action="store_true", help="skip measuring the L2 gather / reduction peaks")
     ap.add_argument("--skip-next-rows", action="store_true",
                     help="skip timing dL/dx, Adam, the fused MLP and the fp16-gradient backward")
+    ap.add_argument("--points", type=int, default=None,
+                    help="encode this many points of the workload instead of all (profiling captures on a "
+                         "reduced batch; the reported line then names a smaller workload than the config's)")
+    ap.add_argument("--min-timed-s", type=float, default=1.0,
+                    help="repeat the K-step loop inside the timed region until it lasts at least this long")
+    ap.add_argument("--stub-step", action="store_true",
+                    help="test the rank plumbing on CPU (gloo, a sleep in place of the GPU step; prints impl=stub)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "b200":
         print("note: fewer than 3 warm-up steps; the timing rules want at least 3", file=sys.stderr)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(args.gpus, argv))
     _, world, _ = dist_env()
     if world != args.gpus:
         print(f"note: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
-    if args.impl == "reference":
+    if args.stub_step:
+        run_stub(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_b200(args)

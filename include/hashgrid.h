@@ -21,8 +21,11 @@
  *   - All array pointers are DEVICE pointers (cudaMalloc'd, or PyTorch CUDA tensors) on the
  *     device that is current when the call is made, unless a parameter says otherwise.
  *     Pointers must be 16-byte aligned; otherwise the call returns HASHGRID_ERR_ALIGN.
- *     Pointers that the CUDA runtime does not report as device-accessible memory are
- *     rejected with HASHGRID_ERR_ARG before anything is launched.
+ *     Host memory (pageable, pinned or registered) and pointers that the CUDA runtime does
+ *     not report as device memory are rejected with HASHGRID_ERR_ARG before anything is
+ *     launched; so is a buffer whose allocation is smaller than the extent the call
+ *     touches. Managed (cudaMallocManaged) memory is accepted when the driver reports its
+ *     allocation's range.
  *   - Layouts (row-major, element offsets):
  *       x          [N, 3]      fp32, x[p*3 + i]; the encoding's domain is [0,1]^3. Points
  *                               outside are not clamped: the same formula applies (int32
@@ -164,13 +167,14 @@ int hashgrid_backward(hashgrid_t h, const float *x, const float *dL_dout, int64_
  * hashgrid_backward_half -- hashgrid_backward into an fp16 gradient table.
  *
  * The same contributions as hashgrid_backward (computed in fp32, merged in fp32 registers
- * by the run walk), rounded to fp16 and reduced with packed 16-byte
- * red.global.add.noftz.v4.f16x2 (round to nearest, subnormals kept): half the gradient
- * memory, and two x-corners share one reduction more often (for F = 2, 3 x-pairs in 4).
- * Each reduction rounds the running sum to fp16, so the result is accurate to about
- * 2^-11 * sqrt(contributions per entry) relative; values beyond fp16 range overflow to
- * infinity. Backward modes: ATOMIC = per-point reductions, every other mode = run
- * merging; the schedule option applies.
+ * by the run walk), rounded to fp16 and reduced with packed fp16 reductions
+ * (red.global.add.noftz f16 / f16x2; round to nearest, subnormals kept): half the gradient
+ * memory. Each reduction rounds the running sum to fp16, so the result is accurate to
+ * about 2^-11 * sqrt(contributions per entry) relative; values beyond fp16 range overflow
+ * to infinity. Backward modes as for hashgrid_backward: ATOMIC = per-point reductions
+ * (16-byte units shared by x-neighbours), RUN_MERGE = run walk with 16-byte units, AUTO and
+ * RUN_LANES = lane-pair run walk (one F-wide reduction per corner; the default), the other
+ * modes = RUN_MERGE; the schedule option applies.
  *
  * x: [N,3] fp32; dL_dout: [N,L*F] fp32; dL_dtable: [L,T,F] fp16 (IEEE binary16),
  * ACCUMULATED into.
@@ -190,7 +194,8 @@ int hashgrid_backward_half(hashgrid_t h, const float *x, const float *dL_dout, i
  * contains x (the one-sided derivative towards +x). fp32 arithmetic, levels summed in order.
  *
  * x: [N,3] fp32; dL_dout: [N,L*F] fp32; table: [L,T,F] of the handle's dtype;
- * dL_dx: [N,3] fp32, OVERWRITTEN. Always point-major (schedule option ignored).
+ * dL_dx: [N,3] fp32, OVERWRITTEN. Always point-major (schedule option ignored); the gather
+ * option selects lane pairs (AUTO, LANES) or one thread per (point, level) (any other).
  */
 int hashgrid_backward_input(hashgrid_t h, const float *x, const float *dL_dout, int64_t N,
                             const void *table, float *dL_dx, void *cuda_stream);
@@ -271,9 +276,13 @@ const char *hashgrid_last_error(void);
  *   HASHGRID_GATHER_PAIR: as SECTOR with 16-byte units: one 128-bit load of the aligned
  *     16-byte unit holding corner (v0, y, z), plus a load of corner (v0 + 1, y, z) when it
  *     is not in that unit (entries wider than 8 bytes load per corner);
- *   HASHGRID_GATHER_AUTO: CORNER (on B200 the L1 already merges the second corner's
- *     request when it falls in the sector just requested, and per-corner loads leave room
- *     for more warps; CORNER measured as fast or faster on every workload tested).
+ *   HASHGRID_GATHER_LANES: two neighbouring threads per (point, level), thread d gathering
+ *     the 4 corners with x offset d, so that each load instruction carries both x-neighbours
+ *     of an edge; the two entries usually share a sector and a line (the x prime is 1), and
+ *     the L1 fetches a shared sector once for both threads. The pair adds its partial sums;
+ *     applies to both schedules;
+ *   HASHGRID_GATHER_AUTO: LANES (measured fastest on every workload: per 2^20 ray samples
+ *     225 us against 250 us for CORNER, per 2^18 uniform points 81 against 95 us).
  * HASHGRID_OPT_BACKWARD_MODE -- how the backward pass reduces into dL_dtable:
  *   HASHGRID_BACKWARD_ATOMIC: each (point, level) reduces its 8 corner contributions, the
  *     two x-corners merged into one 16-byte reduction when they share an aligned unit;
@@ -289,9 +298,13 @@ const char *hashgrid_last_error(void);
  *   HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE: per warp and level, WARP_DEDUP when at least
  *     half of the warp's points lie in a voxel adjacent to the previous point's voxel, else
  *     ATOMIC. Needs F <= 4;
- *   HASHGRID_BACKWARD_AUTO: RUN_MERGE for F <= 4 (measured fastest on samples ordered
- *     along rays, 22% faster than ATOMIC, and within 1-14% of ATOMIC on uniformly scattered
- *     points), ATOMIC for F = 8.
+ *   HASHGRID_BACKWARD_RUN_LANES: RUN_MERGE with two threads per run, thread d keeping the
+ *     sums of the 4 corners with x offset d, each corner reduced on its own (F-wide);
+ *     x-neighbouring corners, which usually share a sector (the x prime is 1), are reduced
+ *     by the same instruction. Needs F <= 4. The schedule option applies;
+ *   HASHGRID_BACKWARD_AUTO: RUN_LANES for F <= 4 (measured fastest on every workload: per
+ *     2^20 ray samples 356 us against 424 us for RUN_MERGE, per 2^22 uniform points 1.74
+ *     against 2.10 ms), ATOMIC for F = 8.
  * HASHGRID_OPT_SCHEDULE -- the order in which (point, level) pairs are visited:
  *   HASHGRID_SCHEDULE_POINT_MAJOR: a block handles all levels of a tile of points (best
  *     when the table fits in L2: the x and upstream-gradient rows are read once and the
@@ -299,8 +312,8 @@ const char *hashgrid_last_error(void);
  *   HASHGRID_SCHEDULE_LEVEL_MAJOR: blocks sweep all points for level 0, then level 1, ...,
  *     so one level's table slice (and gradient slice) stays in L2 while every point
  *     visits it (best for tables much larger than L2; x is read once per level). The
- *     forward pass then gathers per corner, and the warp-dedup backward modes keep their
- *     point-major schedule;
+ *     forward pass then gathers with lane pairs (AUTO, LANES) or per corner (any other
+ *     gather option), and the warp-dedup backward modes keep their point-major schedule;
  *   HASHGRID_SCHEDULE_AUTO: LEVEL_MAJOR when the table is larger than 96 MB, else
  *     POINT_MAJOR.
  * Returns HASHGRID_ERR_ARG for an unknown option or value.
@@ -319,14 +332,16 @@ enum hashgrid_gather {
     HASHGRID_GATHER_AUTO = 0,
     HASHGRID_GATHER_CORNER = 1,
     HASHGRID_GATHER_SECTOR = 2,
-    HASHGRID_GATHER_PAIR = 3
+    HASHGRID_GATHER_PAIR = 3,
+    HASHGRID_GATHER_LANES = 4
 };
 enum hashgrid_backward_mode {
     HASHGRID_BACKWARD_AUTO = 0,
     HASHGRID_BACKWARD_ATOMIC = 1,
     HASHGRID_BACKWARD_WARP_DEDUP = 2,
     HASHGRID_BACKWARD_RUN_MERGE = 3,
-    HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE = 4
+    HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE = 4,
+    HASHGRID_BACKWARD_RUN_LANES = 5
 };
 int hashgrid_set_option(hashgrid_t h, int option, int value);
 int hashgrid_get_option(hashgrid_t h, int option, int *value);

@@ -39,11 +39,21 @@ HASHGRID_GATHER_AUTO = 0
 HASHGRID_GATHER_CORNER = 1
 HASHGRID_GATHER_SECTOR = 2
 HASHGRID_GATHER_PAIR = 3
+HASHGRID_GATHER_LANES = 4
 HASHGRID_BACKWARD_AUTO = 0
 HASHGRID_BACKWARD_ATOMIC = 1
 HASHGRID_BACKWARD_WARP_DEDUP = 2
 HASHGRID_BACKWARD_RUN_MERGE = 3
 HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE = 4
+HASHGRID_BACKWARD_RUN_LANES = 5
+HASHGRID_PROBE_GATHER = 0
+HASHGRID_PROBE_RED = 1
+HASHGRID_PROBE_RED_F16 = 2
+HASHGRID_PROBE_RANDOM = 0
+HASHGRID_PROBE_XPAIR = 1
+HASHGRID_PROBE_SECTOR_PAIR = 2
+HASHGRID_PROBE_LINE_PAIR = 3
+HASHGRID_PROBE_STREAM = 4
 
 
 class HashGridError(RuntimeError):
@@ -76,6 +86,7 @@ def _load() -> ctypes.CDLL:
                                      ctypes.c_float, i32, vp]),
         "hashgrid_mlp_forward": (i32, [vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "hashgrid_debug_indices": (i32, [vp, vp, i64, vp, vp]),
+        "hashgrid_probe": (i32, [i32, i32, i32, vp, sz, i64, vp, ctypes.POINTER(i64), vp]),
         "hashgrid_last_error": (ctypes.c_char_p, []),
         "hashgrid_version": (ctypes.c_char_p, []),
     }
@@ -198,6 +209,16 @@ def hashgrid_mlp_forward(h: int, x, N: int, table, w1, b1, w2, b2, w3, b3, y, de
 
 def hashgrid_debug_indices(h: int, x, N: int, idx_out, stream=None) -> None:
     _check(lib.hashgrid_debug_indices(h, _ptr(x), N, _ptr(idx_out), _stream(stream)))
+
+
+def hashgrid_probe(kind: int, width: int, pattern: int, buf, buf_bytes: int, ops: int, sink=None,
+                   stream=None) -> int:
+    """Runs one memory-system probe (include/hashgrid_probe.h); returns the number of lane
+    operations the kernel performs."""
+    done = ctypes.c_int64()
+    _check(lib.hashgrid_probe(kind, width, pattern, _ptr(buf), buf_bytes, ops, _ptr(sink), ctypes.byref(done),
+                              _stream(stream)))
+    return done.value
 
 
 class HashGrid:

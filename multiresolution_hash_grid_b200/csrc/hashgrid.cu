@@ -22,6 +22,8 @@
 #include "hg_device.cuh"
 #include "hg_mlp.cuh"
 #include "hg_nd.cuh"
+#include "hg_probe.cuh"
+#include "hashgrid_probe.h"
 
 #define HASHGRID_VERSION_STRING "hashgrid-b200 0.1 (sm_100a)"
 
@@ -89,7 +91,9 @@ PFN_memGetAddressRange address_range_fn() {
     return fn;
 }
 
-// Checks one buffer argument that the call will access over [p, p + bytes).
+// Checks one buffer argument that the call will access over [p, p + bytes): not NULL,
+// 16-byte aligned, device memory of the current device or managed memory, and (where the
+// driver reports the allocation's range) the whole extent inside the allocation.
 int check_buffer(const void* p, size_t bytes, const char* name) {
     if (p == nullptr) return fail(HASHGRID_ERR_ARG, "%s is NULL", name);
     if (reinterpret_cast<uintptr_t>(p) % 16 != 0)
@@ -108,23 +112,29 @@ int check_buffer(const void* p, size_t bytes, const char* name) {
         cudaGetLastError();
         return fail(HASHGRID_ERR_CUDA, "cudaGetDevice failed");
     }
-    if (a.type == cudaMemoryTypeDevice) {
-        if (a.device != dev)
-            return fail(HASHGRID_ERR_ARG, "%s lives on device %d but device %d is current", name,
-                        a.device, dev);
-        PFN_memGetAddressRange range = address_range_fn();
-        if (range != nullptr) {
-            CUdeviceptr base = 0;
-            size_t size = 0;
-            if (range(&base, &size, (CUdeviceptr)(uintptr_t)p) == CUDA_SUCCESS) {
-                const uintptr_t end = (uintptr_t)base + size;
-                if ((uintptr_t)p + bytes > end || (uintptr_t)p + bytes < (uintptr_t)p)
-                    return fail(HASHGRID_ERR_ARG,
-                                "%s: the call touches %zu bytes from %p but its allocation ends "
-                                "%zu bytes after it",
-                                name, bytes, p, (size_t)(end - (uintptr_t)p));
-            }
-        }
+    // Host memory (pinned or registered) is device-accessible but its extent cannot be
+    // checked here, and the kernels would read it across the host link: not accepted.
+    if (a.type == cudaMemoryTypeHost)
+        return fail(HASHGRID_ERR_ARG, "%s (%p) is host memory; the library takes device memory", name, p);
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+        return fail(HASHGRID_ERR_ARG, "%s (%p) has unknown memory type %d", name, p, (int)a.type);
+    if (a.type == cudaMemoryTypeDevice && a.device != dev)
+        return fail(HASHGRID_ERR_ARG, "%s lives on device %d but device %d is current", name, a.device, dev);
+    // The extent the call touches must lie inside the pointer's allocation. Device memory
+    // whose range the driver cannot report (none is known) is accepted as before; managed
+    // memory is accepted only when its range is known.
+    PFN_memGetAddressRange range = address_range_fn();
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    const bool known = range != nullptr && range(&base, &size, (CUdeviceptr)(uintptr_t)p) == CUDA_SUCCESS;
+    if (known) {
+        const uintptr_t end = (uintptr_t)base + size;
+        if ((uintptr_t)p + bytes > end || (uintptr_t)p + bytes < (uintptr_t)p)
+            return fail(HASHGRID_ERR_ARG,
+                        "%s: the call touches %zu bytes from %p but its allocation ends %zu bytes after it", name,
+                        bytes, p, (size_t)(end - (uintptr_t)p));
+    } else if (a.type == cudaMemoryTypeManaged) {
+        return fail(HASHGRID_ERR_ARG, "%s (%p): the extent of this managed allocation cannot be checked", name, p);
     }
     return ok();
 }
@@ -172,12 +182,21 @@ int prepare_smem(K kernel, size_t smem) {
 template <int F, typename TT>
 int launch_forward(const hashgrid_s* h, const float* x, int64_t N, const void* table, float* out,
                    int gather, cudaStream_t s) {
+    const size_t smem = hg::tile_smem_bytes(kTile, h->L, F);
+    const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
+    if (gather == hg::kGatherLanes) {
+        auto k = hg::forward_kernel_lanes<F, TT, kTile>;
+        if (int rc = prepare_smem(k, smem)) return rc;
+        // a warp item is 16 points at one level: (kTile / 16) * L items per tile
+        const int items = (kTile / 16) * h->L;
+        const int threads = items * 32 < kMaxThreads ? items * 32 : kMaxThreads;
+        k<<<blocks, threads, smem, s>>>(h->lp, x, N, static_cast<const TT*>(table), out);
+        return launch_status("forward");
+    }
     auto k = gather == hg::kGatherSector ? hg::forward_kernel<F, TT, kTile, hg::kGatherSector>
            : gather == hg::kGatherPair   ? hg::forward_kernel<F, TT, kTile, hg::kGatherPair>
                                          : hg::forward_kernel<F, TT, kTile, hg::kGatherCorner>;
-    const size_t smem = hg::tile_smem_bytes(kTile, h->L, F);
     if (int rc = prepare_smem(k, smem)) return rc;
-    const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
     k<<<blocks, tile_threads(h->L), smem, s>>>(h->lp, x, N, static_cast<const TT*>(table), out);
     return launch_status("forward");
 }
@@ -202,6 +221,25 @@ int launch_backward_mode(const hashgrid_s* h, const float* x, const float* dout,
     return launch_status("backward");
 }
 
+// The forward kernel a handle's gather option selects (AUTO: lane pairs, measured fastest
+// on every workload: per 2^20 ray samples 225 against 250 us per-corner, per 2^18 uniform
+// points 81 against 95 us, fp16 table 1.02 against 1.23 ms per 2^22 points).
+int forward_gather_kernel(const hashgrid_s* h) {
+    switch (h->forward_gather) {
+        case HASHGRID_GATHER_CORNER: return hg::kGatherCorner;
+        case HASHGRID_GATHER_SECTOR: return hg::kGatherSector;
+        case HASHGRID_GATHER_PAIR: return hg::kGatherPair;
+        default: return hg::kGatherLanes;
+    }
+}
+
+// The run walk a handle's backward option selects for F <= 4: lane pairs for AUTO and
+// RUN_LANES (measured 356 against 424 us per 2^20 ray samples, 1.74 against 2.10 ms per
+// 2^22 uniform points), one lane per run for RUN_MERGE.
+bool run_lanes(const hashgrid_s* h) {
+    return h->backward_mode == HASHGRID_BACKWARD_RUN_LANES || h->backward_mode == HASHGRID_BACKWARD_AUTO;
+}
+
 // Level-major when asked, or (AUTO) when the whole table is larger than most of L2.
 constexpr size_t kLevelMajorTableBytes = 96u << 20;
 
@@ -214,17 +252,29 @@ bool level_major(const hashgrid_s* h) {
 
 template <int F, typename TT>
 int launch_forward_levels(const hashgrid_s* h, const float* x, int64_t N, const void* table, float* out,
-                          cudaStream_t s) {
+                          int gather, cudaStream_t s) {
+    if (gather == hg::kGatherLanes) {  // two threads per point
+        const dim3 grid((unsigned)((2 * N + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
+        hg::forward_kernel_levels_lanes<F, TT><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, N, static_cast<const TT*>(table), out);
+        return launch_status("forward");
+    }
     const dim3 grid((unsigned)((N + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
     hg::forward_kernel_levels<F, TT><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, N, static_cast<const TT*>(table), out);
     return launch_status("forward");
 }
 
-// Run merging for every mode but ATOMIC (the warp-dedup modes have no level-major form).
+// Run merging for every mode but ATOMIC (the warp-dedup modes have no level-major form);
+// lane pairs for RUN_LANES.
 template <int F, typename GT>
 int launch_backward_levels(const hashgrid_s* h, const float* x, const float* dout, int64_t N, GT* dtable,
                            cudaStream_t s) {
     if constexpr (F <= 4) {
+        if (run_lanes(h)) {
+            const int64_t runs = (N + hg::kRun - 1) / hg::kRun;
+            const dim3 grid((unsigned)((2 * runs + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
+            hg::backward_kernel_runs_levels_lanes<F, GT><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, dout, N, dtable);
+            return launch_status("backward");
+        }
         if (h->backward_mode != HASHGRID_BACKWARD_ATOMIC) {
             const int64_t runs = (N + hg::kRun - 1) / hg::kRun;
             const dim3 grid((unsigned)((runs + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
@@ -240,7 +290,7 @@ int launch_backward_levels(const hashgrid_s* h, const float* x, const float* dou
 template <int F, typename GT = float>
 int launch_backward_runs(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
                          GT* dtable, cudaStream_t s) {
-    auto k = hg::backward_kernel_runs<F, GT>;
+    auto k = run_lanes(h) ? hg::backward_kernel_runs_lanes<F, GT> : hg::backward_kernel_runs<F, GT>;
     const size_t smem = hg::run_smem_bytes(h->L, F);
     if (int rc = prepare_smem(k, smem)) return rc;
     const unsigned blocks = (unsigned)((N + hg::kRunTile - 1) / hg::kRunTile);
@@ -266,7 +316,8 @@ int launch_backward(const hashgrid_s* h, const float* x, const float* dout, int6
                          h->backward_mode == HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE;
     if (!grouped && level_major(h)) return launch_backward_levels<F, float>(h, x, dout, N, dtable, s);
     if constexpr (F <= 4) {
-        if (h->backward_mode == HASHGRID_BACKWARD_RUN_MERGE || h->backward_mode == HASHGRID_BACKWARD_AUTO)
+        if (h->backward_mode == HASHGRID_BACKWARD_RUN_MERGE || h->backward_mode == HASHGRID_BACKWARD_AUTO ||
+            h->backward_mode == HASHGRID_BACKWARD_RUN_LANES)
             return launch_backward_runs<F>(h, x, dout, N, dtable, s);
         if (h->backward_mode == HASHGRID_BACKWARD_WARP_DEDUP)
             return launch_backward_mode<F, hg::kGroupAlways>(h, x, dout, N, dtable, s);
@@ -276,14 +327,18 @@ int launch_backward(const hashgrid_s* h, const float* x, const float* dout, int6
     return launch_backward_mode<F, hg::kAtomicOnly>(h, x, dout, N, dtable, s);
 }
 
+// dL/dx: lane pairs when the forward gather option asks for them.
 template <int F, typename TT>
 int launch_backward_input(const hashgrid_s* h, const float* x, const float* dout, int64_t N, const void* table,
                           float* dx, cudaStream_t s) {
-    auto k = hg::backward_input_kernel<F, TT, kTile>;
+    const bool lanes = forward_gather_kernel(h) == hg::kGatherLanes;
+    auto k = lanes ? hg::backward_input_kernel_lanes<F, TT, kTile> : hg::backward_input_kernel<F, TT, kTile>;
     const size_t smem = hg::input_grad_smem_bytes(kTile, h->L, F);
     if (int rc = prepare_smem(k, smem)) return rc;
     const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
-    k<<<blocks, tile_threads(h->L), smem, s>>>(h->lp, x, dout, N, static_cast<const TT*>(table), dx);
+    const int items = (kTile / (lanes ? 16 : 32)) * h->L;
+    const int threads = items * 32 < kMaxThreads ? items * 32 : kMaxThreads;
+    k<<<blocks, threads, smem, s>>>(h->lp, x, dout, N, static_cast<const TT*>(table), dx);
     return launch_status("backward_input");
 }
 
@@ -439,7 +494,7 @@ int hashgrid_set_option(hashgrid_t h, int option, int value) {
     if (int rc = check_handle(h)) return rc;
     switch (option) {
         case HASHGRID_OPT_FORWARD_GATHER:
-            if (value < HASHGRID_GATHER_AUTO || value > HASHGRID_GATHER_PAIR)
+            if (value < HASHGRID_GATHER_AUTO || value > HASHGRID_GATHER_LANES)
                 return fail(HASHGRID_ERR_ARG, "forward gather mode %d is not a HASHGRID_GATHER_* value", value);
             h->forward_gather = value;
             return ok();
@@ -449,10 +504,10 @@ int hashgrid_set_option(hashgrid_t h, int option, int value) {
             h->schedule = value;
             return ok();
         case HASHGRID_OPT_BACKWARD_MODE:
-            if (value < HASHGRID_BACKWARD_AUTO || value > HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE)
+            if (value < HASHGRID_BACKWARD_AUTO || value > HASHGRID_BACKWARD_RUN_LANES)
                 return fail(HASHGRID_ERR_ARG, "backward mode %d is not a HASHGRID_BACKWARD_* value", value);
             if ((value == HASHGRID_BACKWARD_WARP_DEDUP || value == HASHGRID_BACKWARD_RUN_MERGE ||
-                 value == HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE) && h->F > 4)
+                 value == HASHGRID_BACKWARD_WARP_DEDUP_ADAPTIVE || value == HASHGRID_BACKWARD_RUN_LANES) && h->F > 4)
                 return fail(HASHGRID_ERR_ARG, "backward mode %d needs F <= 4, F = %d", value, h->F);
             h->backward_mode = value;
             return ok();
@@ -502,15 +557,14 @@ int hashgrid_forward(hashgrid_t h, const float* x, int64_t N, const void* table,
     const bool aligned32 = reinterpret_cast<uintptr_t>(table) % 32 == 0;
     if (h->forward_gather == HASHGRID_GATHER_SECTOR && !aligned32)
         return fail(HASHGRID_ERR_ALIGN, "sector gathers need a 32-byte-aligned table (%p)", table);
-    const int sector = h->forward_gather == HASHGRID_GATHER_SECTOR ? hg::kGatherSector
-                     : h->forward_gather == HASHGRID_GATHER_PAIR   ? hg::kGatherPair
-                                                                   : hg::kGatherCorner;
+    const int sector = forward_gather_kernel(h);
     if (level_major(h)) {
+        const int lg = sector == hg::kGatherLanes ? hg::kGatherLanes : hg::kGatherCorner;
         switch (h->F) {
-            case 1: return half ? launch_forward_levels<1, __half>(h, x, N, table, out, s) : launch_forward_levels<1, float>(h, x, N, table, out, s);
-            case 2: return half ? launch_forward_levels<2, __half>(h, x, N, table, out, s) : launch_forward_levels<2, float>(h, x, N, table, out, s);
-            case 4: return half ? launch_forward_levels<4, __half>(h, x, N, table, out, s) : launch_forward_levels<4, float>(h, x, N, table, out, s);
-            case 8: return half ? launch_forward_levels<8, __half>(h, x, N, table, out, s) : launch_forward_levels<8, float>(h, x, N, table, out, s);
+            case 1: return half ? launch_forward_levels<1, __half>(h, x, N, table, out, lg, s) : launch_forward_levels<1, float>(h, x, N, table, out, lg, s);
+            case 2: return half ? launch_forward_levels<2, __half>(h, x, N, table, out, lg, s) : launch_forward_levels<2, float>(h, x, N, table, out, lg, s);
+            case 4: return half ? launch_forward_levels<4, __half>(h, x, N, table, out, lg, s) : launch_forward_levels<4, float>(h, x, N, table, out, lg, s);
+            case 8: return half ? launch_forward_levels<8, __half>(h, x, N, table, out, lg, s) : launch_forward_levels<8, float>(h, x, N, table, out, lg, s);
         }
     }
     switch (h->F) {
@@ -685,6 +739,64 @@ int hashgrid_debug_indices(hashgrid_t h, const float* x, int64_t N, uint32_t* id
     else
         hg::indices_kernel<<<(unsigned)blocks, threads, 0, s>>>(h->lp, x, N, idx_out);
     return launch_status("debug_indices");
+}
+
+int hashgrid_probe(int kind, int width, int pattern, void* buf, size_t buf_bytes, int64_t ops, float* sink,
+                   int64_t* ops_done, void* cuda_stream) {
+    if (kind != HASHGRID_PROBE_GATHER && kind != HASHGRID_PROBE_RED && kind != HASHGRID_PROBE_RED_F16)
+        return fail(HASHGRID_ERR_ARG, "probe kind %d is not a HASHGRID_PROBE_* kind", kind);
+    const bool red = kind != HASHGRID_PROBE_GATHER;
+    if (!(width == 4 || width == 8 || width == 16 || (width == 32 && !red)))
+        return fail(HASHGRID_ERR_ARG, "probe width %d not supported by this kind", width);
+    if (pattern < HASHGRID_PROBE_RANDOM || pattern > HASHGRID_PROBE_STREAM)
+        return fail(HASHGRID_ERR_ARG, "probe pattern %d is not a HASHGRID_PROBE_* pattern", pattern);
+    if ((pattern == HASHGRID_PROBE_SECTOR_PAIR || pattern == HASHGRID_PROBE_LINE_PAIR) && width != 16)
+        return fail(HASHGRID_ERR_ARG, "the sector- and line-pair patterns take 16-byte units");
+    if (buf_bytes < 256 || (buf_bytes & (buf_bytes - 1)) != 0 || buf_bytes / width > ((size_t)1 << 32))
+        return fail(HASHGRID_ERR_ARG, "probe buffer of %zu bytes: need a power of two from 256 to 2^32 units",
+                    buf_bytes);
+    if (ops < 1) return fail(HASHGRID_ERR_ARG, "ops = %lld must be >= 1", (long long)ops);
+    if (int rc = check_buffer(buf, buf_bytes, "buf")) return rc;
+    if (width == 32 && reinterpret_cast<uintptr_t>(buf) % 32 != 0)
+        return fail(HASHGRID_ERR_ALIGN, "32-byte gathers need a 32-byte-aligned buffer (%p)", buf);
+    if (!red)
+        if (int rc = check_buffer(sink, sizeof(float), "sink")) return rc;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t blocks = (int64_t)sms * 8;
+    const int64_t per_iter = blocks * hg::probe::kThreads * hg::probe::kOpsPerIter;
+    const int64_t iters = (ops + per_iter - 1) / per_iter;
+    if (iters > 0x7fffffffLL) return fail(HASHGRID_ERR_ARG, "ops = %lld is too many", (long long)ops);
+    if (ops_done != nullptr) *ops_done = iters * per_iter;
+    const uint32_t mask = (uint32_t)(buf_bytes / width - 1);
+    char* b = static_cast<char*>(buf);
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    const dim3 grid((unsigned)blocks), block(hg::probe::kThreads);
+    const int it = (int)iters;
+    const uint32_t seed = 0x2545f491u;
+    using namespace hg::probe;
+    if (kind == HASHGRID_PROBE_RED) {
+        switch (width) {
+            case 4: probe_kernel<4, kRedF32><<<grid, block, 0, s>>>(b, mask, pattern, it, seed, sink); break;
+            case 8: probe_kernel<8, kRedF32><<<grid, block, 0, s>>>(b, mask, pattern, it, seed, sink); break;
+            default: probe_kernel<16, kRedF32><<<grid, block, 0, s>>>(b, mask, pattern, it, seed, sink); break;
+        }
+    } else if (kind == HASHGRID_PROBE_RED_F16) {
+        switch (width) {
+            case 4: probe_kernel<4, kRedF16><<<grid, block, 0, s>>>(b, mask, pattern, it, seed, sink); break;
+            case 8: probe_kernel<8, kRedF16><<<grid, block, 0, s>>>(b, mask, pattern, it, seed, sink); break;
+            default: probe_kernel<16, kRedF16><<<grid, block, 0, s>>>(b, mask, pattern, it, seed, sink); break;
+        }
+    } else {
+        switch (width) {
+            case 4: probe_kernel<4, kGather><<<grid, block, 0, s>>>(b, mask, pattern, it, seed, sink); break;
+            case 8: probe_kernel<8, kGather><<<grid, block, 0, s>>>(b, mask, pattern, it, seed, sink); break;
+            case 16: probe_kernel<16, kGather><<<grid, block, 0, s>>>(b, mask, pattern, it, seed, sink); break;
+            default: probe_kernel<32, kGather><<<grid, block, 0, s>>>(b, mask, pattern, it, seed, sink); break;
+        }
+    }
+    return launch_status("probe");
 }
 
 const char* hashgrid_last_error(void) { return g_last_error.c_str(); }

@@ -404,7 +404,7 @@ __host__ __device__ constexpr size_t tile_smem_bytes(int BP, int L, int F) {
 // (needs a 32-byte-aligned table). kGatherPair: the same with 16-byte units (entries of at
 // most 8 bytes; wider entries load per corner).
 // ---------------------------------------------------------------------------------------
-enum GatherMode { kGatherCorner = 0, kGatherSector = 1, kGatherPair = 2 };
+enum GatherMode { kGatherCorner = 0, kGatherSector = 1, kGatherPair = 2, kGatherLanes = 3 };
 
 // 16-byte read-only load.
 __device__ __forceinline__ void ld_unit(const void* p, uint32_t (&w)[4]) {
@@ -559,6 +559,132 @@ __global__ void __launch_bounds__(512, forward_min_blocks(F, kGather)) forward_k
                 o[f] = acc;
             }
             store_smem_entry<F>(os + pl * S + l * F, o);
+        }
+    }
+    __syncthreads();
+    stage_rows_out<(F < 4 ? F : 4)>(os, out, p0, nvalid, W, S);
+}
+
+// ---------------------------------------------------------------------------------------
+// Lane-pair forward (kGatherLanes). The x prime is 1, so a corner and its x-neighbour hash to
+// (v0 ^ K) and ((v0 + 1) ^ K) for the same K: their indices differ only below the lowest
+// carry of v0 + 1, so the two entries share a 32-byte sector most of the time (F = 2 fp32:
+// 3 times in 4) and a 128-byte line almost always (15 times in 16). Here two neighbouring
+// lanes work on one (point, level): lane d0 = lane & 1 gathers the 4 corners whose x offset
+// is d0. Each gather instruction then carries both x-neighbours of 16 cell edges, and the
+// L1 serves a sector (and sends a line request to L2) once for both lanes, where one lane
+// per point loads the two neighbours in different instructions. The pair adds its two
+// partial sums with one shuffle and each lane stores half of the F outputs.
+// ---------------------------------------------------------------------------------------
+struct HalfCorners {
+    uint32_t idx[4];  // corner k: y offset k & 1, z offset k >> 1 (full corner d0 + 2k)
+    float w[4];
+};
+
+// The 4 corners with x offset d0 of one point at one level; weights are the same fp32
+// products, in the same order, as locate_corners computes for those corners.
+__device__ __forceinline__ void locate_half(float x0, float x1, float x2, float scale, uint32_t mask, uint32_t d0,
+                                            HalfCorners& hc) {
+    const float xs0 = __fmul_rn(x0, scale);
+    const float xs1 = __fmul_rn(x1, scale);
+    const float xs2 = __fmul_rn(x2, scale);
+    const int v0 = __float2int_rd(xs0);
+    const int v1 = __float2int_rd(xs1);
+    const int v2 = __float2int_rd(xs2);
+    const float f0 = __fsub_rn(xs0, __int2float_rn(v0));
+    const float f1 = __fsub_rn(xs1, __int2float_rn(v1));
+    const float f2 = __fsub_rn(xs2, __int2float_rn(v2));
+    const uint32_t hx = (uint32_t)v0 + d0;
+    const uint32_t hy0 = (uint32_t)v1 * kPrimeY, hy1 = hy0 + kPrimeY;
+    const uint32_t hz0 = (uint32_t)v2 * kPrimeZ, hz1 = hz0 + kPrimeZ;
+    const float wx = d0 ? f0 : 1.0f - f0;
+    const float wxy[2] = {wx * (1.0f - f1), wx * f1};
+    const float g2 = 1.0f - f2;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        hc.idx[k] = (hx ^ ((k & 1) ? hy1 : hy0) ^ ((k & 2) ? hz1 : hz0)) & mask;
+        hc.w[k] = wxy[k & 1] * ((k & 2) ? f2 : g2);
+    }
+}
+
+// Gathers and interpolates the lane's 4 corners; returns the pair's full sums in o (both
+// lanes get the same values: a + b == b + a in IEEE arithmetic).
+template <int F, typename TT>
+__device__ __forceinline__ void interpolate_pair(const TT* __restrict__ tl, const HalfCorners& hc, unsigned pair,
+                                                 float (&o)[F]) {
+    float e[4][F];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) EntryLoad<F, TT>::load(tl + (uint64_t)hc.idx[k] * F, e[k]);
+#pragma unroll
+    for (int f = 0; f < F; ++f) {
+        float acc = hc.w[0] * e[0][f];
+#pragma unroll
+        for (int k = 1; k < 4; ++k) acc = fmaf(hc.w[k], e[k][f], acc);
+        o[f] = acc + __shfl_xor_sync(pair, acc, 1);
+    }
+}
+
+// Lane d0 of a pair writes outputs [d0 * F/2, (d0 + 1) * F/2) of the (point, level) at p
+// (F = 1: lane 0 writes the one output).
+template <int F, bool kStreaming>
+__device__ __forceinline__ void store_half(float* p, const float (&o)[F], uint32_t d0) {
+    if constexpr (F == 1) {
+        if (d0 == 0) {
+            if constexpr (kStreaming) __stcs(p, o[0]); else *p = o[0];
+        }
+    } else {
+        constexpr int H = F / 2;
+        float v[H];
+#pragma unroll
+        for (int j = 0; j < H; ++j) v[j] = d0 ? o[H + j] : o[j];
+        float* q = p + d0 * H;
+        if constexpr (H == 1) {
+            if constexpr (kStreaming) __stcs(q, v[0]); else *q = v[0];
+        } else if constexpr (H == 2) {
+            const float2 t = make_float2(v[0], v[1]);
+            if constexpr (kStreaming) __stcs(reinterpret_cast<float2*>(q), t); else *reinterpret_cast<float2*>(q) = t;
+        } else {
+            const float4 t = make_float4(v[0], v[1], v[2], v[3]);
+            if constexpr (kStreaming) __stcs(reinterpret_cast<float4*>(q), t); else *reinterpret_cast<float4*>(q) = t;
+        }
+    }
+}
+
+// Lane pairs hold half a point's corners each, so fewer registers than one lane per point:
+// 4 blocks of 512 threads per SM for F <= 2 (<= 32 registers), 3 for F = 4, 2 for F = 8.
+__host__ __device__ constexpr int forward_lanes_min_blocks(int F) { return F <= 2 ? 4 : (F == 4 ? 3 : 2); }
+
+template <int F, typename TT, int BP>
+__global__ void __launch_bounds__(512, forward_lanes_min_blocks(F))
+    forward_kernel_lanes(LevelParams lp, const float* __restrict__ x, int64_t N, const TT* __restrict__ table,
+                         float* __restrict__ out) {
+    extern __shared__ __align__(16) float smem[];
+    const int L = lp.L;
+    const int W = L * F;
+    const int S = W + row_pad(F);
+    float* xs = smem;
+    float* os = smem + BP * 3;
+    const int64_t p0 = (int64_t)blockIdx.x * BP;
+    const int nvalid = (int)min((int64_t)BP, N - p0);
+
+    for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = __ldcs(x + p0 * 3 + i);
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const uint32_t d0 = lane & 1;
+    const unsigned pair = 3u << (lane & 30);
+    const int items = (BP / 16) * L;  // a warp item: 16 points at one level
+    for (int it = warp; it < items; it += nwarps) {
+        const int q = it / L;
+        const int l = it - q * L;
+        const int pl = q * 16 + (lane >> 1);
+        if (pl < nvalid) {  // both lanes of a pair take the same branch
+            HalfCorners hc;
+            locate_half(xs[pl * 3 + 0], xs[pl * 3 + 1], xs[pl * 3 + 2], lp.scale[l], lp.mask, d0, hc);
+            float o[F];
+            interpolate_pair<F, TT>(table + (uint64_t)l * lp.T * F, hc, pair, o);
+            store_half<F, false>(os + pl * S + l * F, o, d0);
         }
     }
     __syncthreads();
@@ -938,6 +1064,198 @@ __global__ void __launch_bounds__(256) backward_kernel_runs(LevelParams lp, cons
 }
 
 // ---------------------------------------------------------------------------------------
+// Lane-pair run walk. As walk_run, but the two lanes of a pair walk one run together: lane
+// d0 = lane & 1 keeps the sums of the 4 corners whose x offset is d0 and reduces them
+// itself, one F-wide reduction per corner. Both lanes see the same points, so they take the
+// same decisions and issue the reductions of x-neighbouring corners in the same
+// instruction. The x prime is 1, so those two entries share a 32-byte sector most of the
+// time, and the L2 serves two reductions into one sector from one instruction faster than
+// two from different instructions (measured on B200 with the probe kernels: 296 against
+// 188 G lane-reductions per second for random 8-byte x-pairs). A step across an x face
+// hands the shared face's 4 sums from one lane to the other with shuffles; y and z steps
+// carry sums inside each lane, as in walk_run.
+// ---------------------------------------------------------------------------------------
+template <int F, typename GT> struct RedLane;
+template <int F> struct RedLane<F, float> {
+    static __device__ __forceinline__ void add(float* p, const float (&v)[F]) { RedAdd<F>::add(p, v); }
+};
+template <> struct RedLane<1, __half> {
+    static __device__ __forceinline__ void add(__half* p, const float (&v)[1]) {
+        const unsigned short h = __half_as_ushort(__float2half_rn(v[0]));
+        asm volatile("red.global.add.noftz.f16 [%0], %1;" ::"l"(p), "h"(h) : "memory");
+    }
+};
+template <> struct RedLane<2, __half> {
+    static __device__ __forceinline__ void add(__half* p, const float (&v)[2]) {
+        __half2 h = __floats2half2_rn(v[0], v[1]);
+        const uint32_t w = *reinterpret_cast<uint32_t*>(&h);
+        asm volatile("red.global.add.noftz.f16x2 [%0], %1;" ::"l"(p), "r"(w) : "memory");
+    }
+};
+template <> struct RedLane<4, __half> {
+    static __device__ __forceinline__ void add(__half* p, const float (&v)[4]) {
+        __half2 a = __floats2half2_rn(v[0], v[1]), b = __floats2half2_rn(v[2], v[3]);
+        const uint32_t wa = *reinterpret_cast<uint32_t*>(&a), wb = *reinterpret_cast<uint32_t*>(&b);
+        asm volatile("red.global.add.noftz.v2.f16x2 [%0], {%1, %2};" ::"l"(p), "r"(wa), "r"(wb) : "memory");
+    }
+};
+
+// locate_half plus the voxel (the walk compares voxels of consecutive points).
+__device__ __forceinline__ void locate_half_voxel(float x0, float x1, float x2, float scale, uint32_t mask,
+                                                  uint32_t d0, HalfCorners& hc, int (&v)[3]) {
+    locate_half(x0, x1, x2, scale, mask, d0, hc);
+    v[0] = __float2int_rd(__fmul_rn(x0, scale));
+    v[1] = __float2int_rd(__fmul_rn(x1, scale));
+    v[2] = __float2int_rd(__fmul_rn(x2, scale));
+}
+
+template <int F, typename GT, class XP, class GL>
+__device__ __forceinline__ void walk_run_pair(GT* dl, float scale, uint32_t mask, int n, uint32_t d0, unsigned pair,
+                                              XP xp, GL gl) {
+    float acc[4][F];
+    uint32_t cidx[4];
+    int cv[3] = {0, 0, 0};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int f = 0; f < F; ++f) acc[k][f] = 0.f;
+    for (int j = 0; j < n; ++j) {
+        float x3[3];
+        xp(j, x3);
+        HalfCorners hc;
+        int v[3];
+        locate_half_voxel(x3[0], x3[1], x3[2], scale, mask, d0, hc, v);
+        float g[F];
+        gl(j, g);
+        if (j > 0) {
+            const int dx = v[0] - cv[0], dy = v[1] - cv[1], dz = v[2] - cv[2];
+            if ((dx | dy | dz) != 0) {
+                const bool face = abs(dx) + abs(dy) + abs(dz) == 1;
+                if (face && dx != 0) {
+                    // x face: the lane on the side left behind reduces its corners and takes
+                    // over its partner's sums (they lie on the shared face); the partner
+                    // starts from zero. dx = +1 leaves x offset 0 behind, dx = -1 offset 1.
+                    const uint32_t leave = dx > 0 ? 0u : 1u;
+                    if (d0 == leave) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) RedLane<F, GT>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+#pragma unroll
+                        for (int f = 0; f < F; ++f) {
+                            const float other = __shfl_xor_sync(pair, acc[k][f], 1);
+                            acc[k][f] = d0 == leave ? other : 0.f;
+                        }
+                } else if (face) {
+                    // y or z face: corner bit b (0: y, 1: z) of the local corner number k;
+                    // corners whose offset along the step's axis is leave_bit are left behind,
+                    // the new corners with that offset take the sums of their face neighbours
+                    const int b = dy != 0 ? 0 : 1;
+                    const uint32_t leave_bit = (dy + dz) > 0 ? 0u : 1u;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if ((((uint32_t)k >> b) & 1u) == leave_bit)
+                            RedLane<F, GT>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
+                    float old[4][F];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+#pragma unroll
+                        for (int f = 0; f < F; ++f) old[k][f] = acc[k][f];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const bool keep = (((uint32_t)k >> b) & 1u) == leave_bit;
+#pragma unroll
+                        for (int f = 0; f < F; ++f) acc[k][f] = keep ? (b == 0 ? old[k ^ 1][f] : old[k ^ 2][f]) : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        RedLane<F, GT>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
+#pragma unroll
+                        for (int f = 0; f < F; ++f) acc[k][f] = 0.f;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            cidx[k] = hc.idx[k];
+#pragma unroll
+            for (int f = 0; f < F; ++f) acc[k][f] = fmaf(hc.w[k], g[f], acc[k][f]);
+        }
+        cv[0] = v[0];
+        cv[1] = v[1];
+        cv[2] = v[2];
+    }
+    if (n > 0) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) RedLane<F, GT>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
+    }
+}
+
+// Block: kRunTile points (32 runs of kRun) and 8 warps, shared memory as backward_kernel_runs;
+// a warp item is 16 runs at one level (a lane pair per run).
+template <int F, typename GT>
+__global__ void __launch_bounds__(256) backward_kernel_runs_lanes(LevelParams lp, const float* __restrict__ x,
+                                                                 const float* __restrict__ dout, int64_t N,
+                                                                 GT* __restrict__ dtable) {
+    static_assert(F <= 4, "run merging keeps 4 x F sums per lane in registers");
+    extern __shared__ __align__(16) float smem[];
+    const int L = lp.L;
+    const int W = L * F;
+    const int S = run_row_stride(L, F);
+    const int G = run_g_stride(L, F);
+    constexpr int XS = run_x_stride();
+    float* xs = smem;
+    float* gs = smem + 32 * XS;
+    const int64_t p0 = (int64_t)blockIdx.x * kRunTile;
+    const int nvalid = (int)min((int64_t)kRunTile, N - p0);
+
+    for (int k = threadIdx.x; k < nvalid * 3; k += blockDim.x) {
+        const int p = k / 3, i = k - 3 * (k / 3);
+        xs[(p / kRun) * XS + (p % kRun) * 3 + i] = __ldcs(x + p0 * 3 + k);
+    }
+    {
+        constexpr int V = F < 4 ? F : 4;
+        const int per_row = W / V;
+        const float* base = dout + p0 * (int64_t)W;
+        for (int k = threadIdx.x; k < nvalid * per_row; k += blockDim.x) {
+            const int row = k / per_row;
+            const int col = (k - row * per_row) * V;
+            float* dst = gs + (row / kRun) * G + (row % kRun) * S + col;
+            const float* src = base + (int64_t)row * W + col;
+            if constexpr (V == 4) {
+                *reinterpret_cast<float4*>(dst) = __ldcs(reinterpret_cast<const float4*>(src));
+            } else if constexpr (V == 2) {
+                *reinterpret_cast<float2*>(dst) = __ldcs(reinterpret_cast<const float2*>(src));
+            } else {
+                *dst = __ldcs(src);
+            }
+        }
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const uint32_t d0 = lane & 1;
+    const unsigned pair = 3u << (lane & 30);
+    for (int it = warp; it < 2 * L; it += nwarps) {
+        const int h = it / L;
+        const int l = it - h * L;
+        const int run = h * 16 + (lane >> 1);
+        const int jmax = min(kRun, nvalid - run * kRun);  // the same for both lanes of a pair
+        GT* dl = dtable + (uint64_t)l * lp.T * F;
+        walk_run_pair<F>(dl, lp.scale[l], lp.mask, jmax, d0, pair,
+                         [&](int j, float* x3) {
+                             const float* q = xs + run * XS + j * 3;
+                             x3[0] = q[0]; x3[1] = q[1]; x3[2] = q[2];
+                         },
+                         [&](int j, float* g) { load_smem_entry<F>(gs + run * G + j * S + l * F, g); });
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // Level-major schedules, for tables larger than L2. Grid (tiles, L): blocks are issued with
 // the tile index fastest, so the GPU works through the levels one after another and the
 // current level's table slice (backward: its gradient slice) stays resident in L2 while
@@ -1044,6 +1362,35 @@ __global__ void __launch_bounds__(kLevelBlock) forward_kernel_levels(LevelParams
     store_global_entry<F>(out + p * (int64_t)(lp.L * F) + l * F, o);
 }
 
+// Level-major forward with lane pairs: two threads per point at level blockIdx.y.
+template <int F, typename TT>
+__global__ void __launch_bounds__(kLevelBlock) forward_kernel_levels_lanes(LevelParams lp, const float* __restrict__ x,
+                                                                          int64_t N, const TT* __restrict__ table,
+                                                                          float* __restrict__ out) {
+    const int l = blockIdx.y;
+    const int64_t p = ((int64_t)blockIdx.x * kLevelBlock + threadIdx.x) >> 1;
+    if (p >= N) return;  // both lanes of a pair return together
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t d0 = lane & 1;
+    const unsigned pair = 3u << (lane & 30);
+    HalfCorners hc;
+    locate_half(__ldcs(x + p * 3), __ldcs(x + p * 3 + 1), __ldcs(x + p * 3 + 2), lp.scale[l], lp.mask, d0, hc);
+    const TT* tl = table + (uint64_t)l * lp.T * F;
+    const uint64_t pol = l2_evict_last_policy();
+    float e[4][F];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) load_entry_policy<F, TT>(tl + (uint64_t)hc.idx[k] * F, e[k], pol);
+    float o[F];
+#pragma unroll
+    for (int f = 0; f < F; ++f) {
+        float acc = hc.w[0] * e[0][f];
+#pragma unroll
+        for (int k = 1; k < 4; ++k) acc = fmaf(hc.w[k], e[k][f], acc);
+        o[f] = acc + __shfl_xor_sync(pair, acc, 1);
+    }
+    store_half<F, true>(out + p * (int64_t)(lp.L * F) + l * F, o, d0);
+}
+
 template <int F, typename GT>
 __global__ void __launch_bounds__(kLevelBlock) backward_kernel_atomic_levels(LevelParams lp, const float* __restrict__ x,
                                                                             const float* __restrict__ dout, int64_t N,
@@ -1085,6 +1432,28 @@ __global__ void __launch_bounds__(kLevelBlock) backward_kernel_runs_levels(Level
                     x3[0] = __ldcs(q); x3[1] = __ldcs(q + 1); x3[2] = __ldcs(q + 2);
                 },
                 [&](int j, float* g) { load_global_entry<F>(dout + (p0 + j) * W + l * F, g); });
+}
+
+// Level-major lane-pair run walk: two threads per run of kRun consecutive points at level
+// blockIdx.y.
+template <int F, typename GT>
+__global__ void __launch_bounds__(kLevelBlock) backward_kernel_runs_levels_lanes(LevelParams lp,
+                                                                                const float* __restrict__ x,
+                                                                                const float* __restrict__ dout,
+                                                                                int64_t N, GT* __restrict__ dtable) {
+    const int l = blockIdx.y;
+    const int64_t p0 = (((int64_t)blockIdx.x * kLevelBlock + threadIdx.x) >> 1) * kRun;
+    if (p0 >= N) return;  // both lanes of a pair return together
+    const int n = (int)min((int64_t)kRun, N - p0);
+    const int64_t W = lp.L * F;
+    const uint32_t lane = threadIdx.x & 31;
+    GT* dl = dtable + (uint64_t)l * lp.T * F;
+    walk_run_pair<F>(dl, lp.scale[l], lp.mask, n, lane & 1, 3u << (lane & 30),
+                     [&](int j, float* x3) {
+                         const float* q = x + (p0 + j) * 3;
+                         x3[0] = __ldcs(q); x3[1] = __ldcs(q + 1); x3[2] = __ldcs(q + 2);
+                     },
+                     [&](int j, float* g) { load_global_entry<F>(dout + (p0 + j) * W + l * F, g); });
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1162,6 +1531,86 @@ __global__ void __launch_bounds__(512, F <= 2 ? 3 : 2) backward_input_kernel(Lev
             pp[0] = n * d0;
             pp[1] = n * d1;
             pp[2] = n * d2;
+        }
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < nvalid * 3; t += blockDim.x) {  // t = 3 * point + axis
+        float s = 0.f;
+        for (int l = 0; l < L; ++l) s += part[(size_t)l * BP * 3 + t];
+        __stcs(dx + p0 * 3 + t, s);
+    }
+}
+
+// dL/dx with lane pairs (as forward_kernel_lanes): lane d0 gathers the 4 corners with x
+// offset d0, forms its share of the three weight-derivative sums, and the pair adds them
+// with shuffles.
+template <int F, typename TT, int BP>
+__global__ void __launch_bounds__(512, F <= 2 ? 3 : 2) backward_input_kernel_lanes(LevelParams lp,
+                                                                               const float* __restrict__ x,
+                                                                               const float* __restrict__ dout,
+                                                                               int64_t N, const TT* __restrict__ table,
+                                                                               float* __restrict__ dx) {
+    extern __shared__ __align__(16) float smem[];
+    const int L = lp.L;
+    const int W = L * F;
+    const int S = W + row_pad(F);
+    float* xs = smem;
+    float* gs = smem + BP * 3;
+    float* part = gs + BP * S;  // [L][BP][3]
+    const int64_t p0 = (int64_t)blockIdx.x * BP;
+    const int nvalid = (int)min((int64_t)BP, N - p0);
+
+    for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = __ldcs(x + p0 * 3 + i);
+    stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    const uint32_t d0 = lane & 1;
+    const unsigned pair = 3u << (lane & 30);
+    const int items = (BP / 16) * L;
+    for (int it = warp; it < items; it += nwarps) {
+        const int q = it / L;
+        const int l = it - q * L;
+        const int pl = q * 16 + (lane >> 1);
+        if (pl < nvalid) {  // both lanes of a pair take the same branch
+            const float x0 = xs[pl * 3 + 0], x1 = xs[pl * 3 + 1], x2 = xs[pl * 3 + 2];
+            const float scale = lp.scale[l];
+            HalfCorners hc;
+            locate_half(x0, x1, x2, scale, lp.mask, d0, hc);
+            const float xs0 = __fmul_rn(x0, scale), xs1 = __fmul_rn(x1, scale), xs2 = __fmul_rn(x2, scale);
+            const float f0 = __fsub_rn(xs0, __int2float_rn(__float2int_rd(xs0)));
+            const float f1 = __fsub_rn(xs1, __int2float_rn(__float2int_rd(xs1)));
+            const float f2 = __fsub_rn(xs2, __int2float_rn(__float2int_rd(xs2)));
+            const TT* tl = table + (uint64_t)l * lp.T * F;
+            float e[4][F];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) EntryLoad<F, TT>::load(tl + (uint64_t)hc.idx[k] * F, e[k]);
+            float g[F];
+            load_smem_entry<F>(gs + pl * S + l * F, g);
+            const float w0 = d0 ? f0 : 1.0f - f0;
+            const float w1[2] = {1.0f - f1, f1};
+            const float w2[2] = {1.0f - f2, f2};
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int b1 = k & 1, b2 = k >> 1;
+                float sc = g[0] * e[k][0];
+#pragma unroll
+                for (int f = 1; f < F; ++f) sc = fmaf(g[f], e[k][f], sc);
+                const float s0 = d0 ? sc : -sc;
+                const float s1 = b1 ? sc : -sc;
+                const float s2 = b2 ? sc : -sc;
+                a0 = fmaf(s0, w1[b1] * w2[b2], a0);
+                a1 = fmaf(s1, w0 * w2[b2], a1);
+                a2 = fmaf(s2, w0 * w1[b1], a2);
+            }
+            a0 += __shfl_xor_sync(pair, a0, 1);
+            a1 += __shfl_xor_sync(pair, a1, 1);
+            a2 += __shfl_xor_sync(pair, a2, 1);
+            float* pp = part + ((size_t)l * BP + pl) * 3;
+            pp[d0] = scale * (d0 ? a1 : a0);
+            if (d0 == 0) pp[2] = scale * a2;
         }
     }
     __syncthreads();

@@ -3,6 +3,7 @@ exports every function that include/hashgrid.h declares, handles report their pa
 the library's resolution schedule agrees with the oracle's and with exact integer floors,
 and invalid arguments are rejected with the documented status before any launch."""
 import ctypes
+import glob
 import os
 import re
 import shutil
@@ -22,15 +23,19 @@ HEADER = os.path.join(INCLUDE_DIR, "hashgrid.h")
 LIB_PATH = os.path.join(ROOT, "multiresolution_hash_grid_b200", "libhashgrid.so")
 
 
-def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(hashgrid_\w+)\s*\(", text)))
+def declared_functions(headers=None):
+    """Every hashgrid_* function declared in include/*.h (comments stripped)."""
+    names = set()
+    for path in headers or sorted(glob.glob(os.path.join(INCLUDE_DIR, "*.h"))):
+        text = re.sub(r"/\*.*?\*/", "", open(path).read(), flags=re.S)
+        names |= set(re.findall(r"\b(hashgrid_\w+)\s*\(", text))
+    return sorted(names)
 
 
 def test_library_exports_every_declared_function():
     names = declared_functions()
     assert "hashgrid_forward" in names and "hashgrid_backward" in names and "hashgrid_create" in names
+    assert "hashgrid_probe" in names
     lib = ctypes.CDLL(hg.LIB_PATH)
     missing = [n for n in names if not hasattr(lib, n)]
     assert not missing, missing
@@ -127,7 +132,7 @@ def test_options():
         assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_SCHEDULE) == hg.HASHGRID_SCHEDULE_AUTO
         hg.hashgrid_set_option(h, hg.HASHGRID_OPT_SCHEDULE, hg.HASHGRID_SCHEDULE_LEVEL_MAJOR)
         assert hg.hashgrid_get_option(h, hg.HASHGRID_OPT_SCHEDULE) == hg.HASHGRID_SCHEDULE_LEVEL_MAJOR
-        for opt, val in [(hg.HASHGRID_OPT_SCHEDULE, 3), (hg.HASHGRID_OPT_FORWARD_GATHER, 4), (hg.HASHGRID_OPT_BACKWARD_MODE, -1), (hg.HASHGRID_OPT_BACKWARD_MODE, 5), (7, 0)]:
+        for opt, val in [(hg.HASHGRID_OPT_SCHEDULE, 3), (hg.HASHGRID_OPT_FORWARD_GATHER, 5), (hg.HASHGRID_OPT_BACKWARD_MODE, -1), (hg.HASHGRID_OPT_BACKWARD_MODE, 6), (7, 0)]:
             assert hg.lib.hashgrid_set_option(h, opt, val) == hg.HASHGRID_ERR_ARG
         assert hg.lib.hashgrid_set_option(None, 0, 0) == hg.HASHGRID_ERR_ARG
     finally:
@@ -136,6 +141,7 @@ def test_options():
     try:   # warp dedup works on 16-byte gradient units: F <= 4 only
         assert hg.lib.hashgrid_set_option(h8, hg.HASHGRID_OPT_BACKWARD_MODE, hg.HASHGRID_BACKWARD_WARP_DEDUP) == hg.HASHGRID_ERR_ARG
         assert hg.lib.hashgrid_set_option(h8, hg.HASHGRID_OPT_BACKWARD_MODE, hg.HASHGRID_BACKWARD_RUN_MERGE) == hg.HASHGRID_ERR_ARG
+        assert hg.lib.hashgrid_set_option(h8, hg.HASHGRID_OPT_BACKWARD_MODE, hg.HASHGRID_BACKWARD_RUN_LANES) == hg.HASHGRID_ERR_ARG
     finally:
         hg.hashgrid_destroy(h8)
 
@@ -205,6 +211,7 @@ def test_binding_fails_loudly_without_library(tmp_path):
 C_CLIENT = r"""
 #include <stdio.h>
 #include "hashgrid.h"
+#include "hashgrid_probe.h"
 
 int main(void)
 {
@@ -219,6 +226,7 @@ int main(void)
     if (hashgrid_table_elems(h) != (size_t)16 * 524288 * 2 || hashgrid_output_width(h) != 32) return 4;
     /* an invalid call is an error code before any launch, with a message */
     if (hashgrid_forward(h, NULL, 4, NULL, NULL, NULL) == HASHGRID_OK || hashgrid_last_error()[0] == 0) return 5;
+    if (hashgrid_probe(7, 8, HASHGRID_PROBE_RANDOM, NULL, 1024, 1, NULL, NULL, NULL) != HASHGRID_ERR_ARG) return 6;
     hashgrid_destroy(h);
     printf("%s\n", hashgrid_version());
     return 0;
@@ -228,7 +236,7 @@ int main(void)
 
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc missing")
 def test_header_is_plain_c_and_links(tmp_path):
-    """A C99 client compiled with gcc -Wall -Werror against include/hashgrid.h links to the
+    """A C99 client compiled with gcc -Wall -Werror against include/*.h links to the
     library and uses it without a GPU (create, queries, an argument error, destroy)."""
     src = tmp_path / "client.c"
     src.write_text(C_CLIENT)

@@ -1,8 +1,11 @@
 """Multi-rank host logic of the benchmark, on CPU with the gloo backend (world size 2):
 the max-over-ranks timing reduction, the barrier, per-rank batches and the whole-job
 rate. The data path itself has no collective: each rank encodes its own points."""
+import json
 import os
 import socket
+import subprocess
+import sys
 
 import pytest
 import torch.multiprocessing as mp
@@ -80,3 +83,28 @@ def test_cpu_oracle_timers():
     assert rows["backward_input"]["value"] > 0
     assert rows["adam_step"]["value"] > 0 and rows["adam_step"]["unit"] == "elements/s"
     assert "mlp_forward" not in rows   # L*F = 8 has no MLP
+
+
+@pytest.mark.timeout(180)
+def test_gpus_flag_starts_that_many_ranks():
+    """``bench.py --gpus 2`` without a launcher starts two ranks itself (torch.distributed.run
+    on 127.0.0.1); with the CPU stub step in place of the GPU work they rendezvous over gloo
+    and rank 0 alone prints one line that reports both ranks."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--steps", "4", "--warmup", "3", "--stub-step"],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=170)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "stub" and line["n_gpus"] == 2 and line["steps"] == 4
+    # rank 1 sleeps twice as long per step: the slowest rank sets the time
+    assert line["ms_per_step"] >= 4.0
+    assert line["value"] == pytest.approx(2 * (1 << 20) / (line["ms_per_step"] * 1e-3), rel=1e-2)
+
+
+def test_loop_repeats():
+    assert bench.loop_repeats(20, 0.7e-3, 1.0) == 72      # 20 steps x 0.7 ms -> 72 loops >= 1 s
+    assert bench.loop_repeats(20, 0.1, 1.0) == 1
+    assert bench.loop_repeats(20, 0.7e-3, 0.0) == 1
