@@ -15,7 +15,10 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libhashgrid.so")
+# HASHGRID_CHECKED=1 loads the checked build (every global access of the kernels range-checked,
+# violations returned as HASHGRID_ERR_DEVICE_CHECK; synchronous, for testing).
+CHECKED = os.environ.get("HASHGRID_CHECKED", "0") not in ("", "0")
+LIB_PATH = os.path.join(HERE, "libhashgrid_checked.so" if CHECKED else "libhashgrid.so")
 
 HASHGRID_F32 = 0
 HASHGRID_F16 = 1
@@ -64,7 +67,8 @@ class HashGridError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built: run `python multiresolution_hash_grid_b200/build.py`")
+        raise ImportError(f"{LIB_PATH} is not built: run `python multiresolution_hash_grid_b200/build.py"
+                          f"{' --checked' if CHECKED else ''}`")
     lib = ctypes.CDLL(LIB_PATH)
     i32, i64, vp, sz = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
     protos = {

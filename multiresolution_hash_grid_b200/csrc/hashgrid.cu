@@ -13,7 +13,9 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
+#include <initializer_list>
 #include <new>
 #include <string>
 #include <type_traits>
@@ -25,7 +27,11 @@
 #include "hg_probe.cuh"
 #include "hashgrid_probe.h"
 
-#define HASHGRID_VERSION_STRING "hashgrid-b200 0.1 (sm_100a)"
+#ifdef HASHGRID_CHECKED
+#define HASHGRID_VERSION_STRING "hashgrid-b200 0.2 (sm_100a, checked)"
+#else
+#define HASHGRID_VERSION_STRING "hashgrid-b200 0.2 (sm_100a)"
+#endif
 
 struct hashgrid_s {
     int D;  // input dimensions (3 for hashgrid_create)
@@ -327,18 +333,31 @@ int launch_backward(const hashgrid_s* h, const float* x, const float* dout, int6
     return launch_backward_mode<F, hg::kAtomicOnly>(h, x, dout, N, dtable, s);
 }
 
-// dL/dx: lane pairs when the forward gather option asks for them.
+// dL/dx: warp-owned lane pairs when the gather option selects lane pairs (AUTO, LANES),
+// else one thread per (point, level). A warp stages its 16 upstream-gradient rows: 16 warps
+// per block for rows of up to 64 floats, 4 above (shared memory).
+template <int F, typename TT, int kW>
+int launch_backward_input_warp(const hashgrid_s* h, const float* x, const float* dout, int64_t N, const void* table,
+                               float* dx, cudaStream_t s) {
+    auto k = hg::backward_input_kernel_warp<F, TT, kW>;
+    const size_t smem = sizeof(float) * (size_t)kW * hg::kWarpPoints * (h->L * F + hg::row_pad(F));
+    if (int rc = prepare_smem(k, smem)) return rc;
+    const int64_t pts = (int64_t)kW * hg::kWarpPoints;
+    k<<<(unsigned)((N + pts - 1) / pts), 32 * kW, smem, s>>>(h->lp, x, dout, N, static_cast<const TT*>(table), dx);
+    return launch_status("backward_input");
+}
+
 template <int F, typename TT>
 int launch_backward_input(const hashgrid_s* h, const float* x, const float* dout, int64_t N, const void* table,
                           float* dx, cudaStream_t s) {
-    const bool lanes = forward_gather_kernel(h) == hg::kGatherLanes;
-    auto k = lanes ? hg::backward_input_kernel_lanes<F, TT, kTile> : hg::backward_input_kernel<F, TT, kTile>;
+    if (forward_gather_kernel(h) == hg::kGatherLanes)
+        return h->L * F <= 64 ? launch_backward_input_warp<F, TT, 16>(h, x, dout, N, table, dx, s)
+                              : launch_backward_input_warp<F, TT, 4>(h, x, dout, N, table, dx, s);
+    auto k = hg::backward_input_kernel<F, TT, kTile>;
     const size_t smem = hg::input_grad_smem_bytes(kTile, h->L, F);
     if (int rc = prepare_smem(k, smem)) return rc;
     const unsigned blocks = (unsigned)((N + kTile - 1) / kTile);
-    const int items = (kTile / (lanes ? 16 : 32)) * h->L;
-    const int threads = items * 32 < kMaxThreads ? items * 32 : kMaxThreads;
-    k<<<blocks, threads, smem, s>>>(h->lp, x, dout, N, static_cast<const TT*>(table), dx);
+    k<<<blocks, tile_threads(h->L), smem, s>>>(h->lp, x, dout, N, static_cast<const TT*>(table), dx);
     return launch_status("backward_input");
 }
 
@@ -346,7 +365,10 @@ template <int F, typename TT, int K1>
 int launch_mlp_forward(const hashgrid_s* h, const float* x, int64_t N, const void* table, const void* w1,
                        const float* b1, const void* w2, const float* b2, const void* w3, const float* b3, float* y,
                        int* status, cudaStream_t s) {
-    auto k = hg::mlp::mlp_forward_kernel<F, TT, K1>;
+    // lane-pair producers when the gather option selects lane pairs (F <= 4)
+    constexpr bool kCanLanes = F <= 4;
+    const bool lanes = kCanLanes && forward_gather_kernel(h) == hg::kGatherLanes;
+    auto k = lanes ? hg::mlp::mlp_forward_kernel<F, TT, K1, kCanLanes> : hg::mlp::mlp_forward_kernel<F, TT, K1, false>;
     const size_t smem = hg::mlp::ws_smem_bytes(K1);
     if (int rc = prepare_smem(k, smem)) return rc;
     int dev = 0, sms = 148, smem_sm = 0;
@@ -361,7 +383,7 @@ int launch_mlp_forward(const hashgrid_s* h, const float* x, int64_t N, const voi
     const int64_t tiles = (N + hg::mlp::kM - 1) / hg::mlp::kM;
     const int64_t cap = (int64_t)sms * per_sm;
     const unsigned blocks = (unsigned)(tiles < cap ? tiles : cap);
-    k<<<blocks, hg::mlp::block_threads(F), smem, s>>>(h->lp, x, N, static_cast<const TT*>(table),
+    k<<<blocks, hg::mlp::block_threads(F, lanes), smem, s>>>(h->lp, x, N, static_cast<const TT*>(table),
                                                static_cast<const uint16_t*>(w1), b1, static_cast<const uint16_t*>(w2),
                                                b2, static_cast<const uint16_t*>(w3), b3, y, status);
     return launch_status("mlp_forward");
@@ -420,6 +442,71 @@ int nd_dispatch(const hashgrid_s* h, Fn&& fn) {
     HG_ND_CASE(4, 1) HG_ND_CASE(4, 2) HG_ND_CASE(4, 4) HG_ND_CASE(4, 8)
 #undef HG_ND_CASE
     return fail(HASHGRID_ERR_ARG, "corrupt handle");
+}
+
+// Buffers of one call for the checked build's range checks: (role, base, bytes).
+struct CheckBuf {
+    int role;
+    const void* p;
+    size_t bytes;
+};
+
+// Runs fn (the call's launches). In the checked build (HASHGRID_CHECKED) the byte ranges
+// of the call's buffers are first recorded for the kernels' range checks (roles the call
+// does not use stay unrestricted), and after the launches the device status word is read
+// back on the call's stream: a tripped check is cleared and reported as
+// HASHGRID_ERR_DEVICE_CHECK. Calls are then synchronous, and calls running at the same
+// time on several streams would share the recorded ranges: the checked build is for one
+// stream at a time. In the regular build this only calls fn.
+template <class Fn>
+int run_checked(cudaStream_t s, std::initializer_list<CheckBuf> bufs, const char* what, Fn&& fn) {
+#ifdef HASHGRID_CHECKED
+    hg::CheckRanges r;
+    for (int i = 0; i < hg::kChkRoles; ++i) {
+        r.lo[i] = 0;
+        r.hi[i] = ~0ull;
+    }
+    for (const CheckBuf& b : bufs) {
+        r.lo[b.role] = (uint64_t)(uintptr_t)b.p;
+        r.hi[b.role] = (uint64_t)(uintptr_t)b.p + b.bytes;
+    }
+    // Test hook: HASHGRID_CHECK_SHRINK_OUT=n records the output buffer n bytes shorter than
+    // it is, so that a test can make the checks trip on accesses that still lie inside the
+    // caller's buffer.
+    if (const char* shrink = std::getenv("HASHGRID_CHECK_SHRINK_OUT")) {
+        const uint64_t n = std::strtoull(shrink, nullptr, 10);
+        if (r.hi[hg::kChkOut] != ~0ull) r.hi[hg::kChkOut] -= std::min<uint64_t>(n, r.hi[hg::kChkOut] - r.lo[hg::kChkOut]);
+    }
+    if (cudaMemcpyToSymbolAsync(hg::g_check_ranges, &r, sizeof r, 0, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(HASHGRID_ERR_CUDA, "%s: recording the checked ranges failed", what);
+    }
+    const int rc = fn();
+    if (rc != HASHGRID_OK) return rc;
+    unsigned int flags = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&flags, hg::g_check_flags, sizeof flags, 0, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(HASHGRID_ERR_CUDA, "%s: reading the device status failed: %s", what, cudaGetErrorString(e));
+    }
+    if (flags != 0) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(hg::g_check_flags, &zero, sizeof zero);
+        static const char* names[hg::kChkRoles] = {"x", "table", "output", "dL_dout", "dL_dtable", "adam_m", "adam_v"};
+        std::string which;
+        for (int i = 0; i < hg::kChkRoles; ++i)
+            if (flags & (1u << i)) which += std::string(which.empty() ? "" : ", ") + names[i];
+        return fail(HASHGRID_ERR_DEVICE_CHECK, "%s: a device range check tripped on %s (the access was skipped)", what,
+                    which.c_str());
+    }
+    return rc;
+#else
+    (void)s;
+    (void)bufs;
+    (void)what;
+    return fn();
+#endif
 }
 
 size_t table_bytes(const hashgrid_s* h) {
@@ -547,6 +634,9 @@ int hashgrid_forward(hashgrid_t h, const float* x, int64_t N, const void* table,
     if (int rc = check_buffer(table, table_bytes(h), "table")) return rc;
     if (int rc = check_buffer(out, (size_t)N * W * sizeof(float), "out")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    return run_checked(s, {{hg::kChkX, x, (size_t)N * h->D * sizeof(float)}, {hg::kChkTable, table, table_bytes(h)},
+                           {hg::kChkOut, out, (size_t)N * W * sizeof(float)}},
+                       "forward", [&]() -> int {
     const bool half = h->dtype == HASHGRID_F16;
     if (h->D != 3)
         return nd_dispatch(h, [&](auto d, auto f) {
@@ -574,6 +664,7 @@ int hashgrid_forward(hashgrid_t h, const float* x, int64_t N, const void* table,
         case 8: return half ? launch_forward<8, __half>(h, x, N, table, out, sector, s) : launch_forward<8, float>(h, x, N, table, out, sector, s);
     }
     return fail(HASHGRID_ERR_ARG, "corrupt handle");
+    });
 }
 
 int hashgrid_backward(hashgrid_t h, const float* x, const float* dL_dout, int64_t N, float* dL_dtable,
@@ -586,6 +677,9 @@ int hashgrid_backward(hashgrid_t h, const float* x, const float* dL_dout, int64_
     if (int rc = check_buffer(dL_dout, (size_t)N * W * sizeof(float), "dL_dout")) return rc;
     if (int rc = check_buffer(dL_dtable, hashgrid_table_elems(h) * sizeof(float), "dL_dtable")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    return run_checked(s, {{hg::kChkX, x, (size_t)N * h->D * sizeof(float)}, {hg::kChkDout, dL_dout, (size_t)N * W * sizeof(float)},
+                           {hg::kChkGrad, dL_dtable, hashgrid_table_elems(h) * sizeof(float)}},
+                       "backward", [&]() -> int {
     if (h->D != 3)
         return nd_dispatch(h, [&](auto d, auto f) {
             return launch_nd_backward<decltype(d)::value, decltype(f)::value, float>(h, x, dL_dout, N, dL_dtable, s);
@@ -597,6 +691,7 @@ int hashgrid_backward(hashgrid_t h, const float* x, const float* dL_dout, int64_
         case 8: return launch_backward<8>(h, x, dL_dout, N, dL_dtable, s);
     }
     return fail(HASHGRID_ERR_ARG, "corrupt handle");
+    });
 }
 
 int hashgrid_backward_half(hashgrid_t h, const float* x, const float* dL_dout, int64_t N, void* dL_dtable,
@@ -610,6 +705,9 @@ int hashgrid_backward_half(hashgrid_t h, const float* x, const float* dL_dout, i
     if (int rc = check_buffer(dL_dtable, hashgrid_table_elems(h) * 2, "dL_dtable")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     __half* d = static_cast<__half*>(dL_dtable);
+    return run_checked(s, {{hg::kChkX, x, (size_t)N * h->D * sizeof(float)}, {hg::kChkDout, dL_dout, (size_t)N * W * sizeof(float)},
+                           {hg::kChkGrad, dL_dtable, hashgrid_table_elems(h) * 2}},
+                       "backward_half", [&]() -> int {
     if (h->D != 3)
         return nd_dispatch(h, [&](auto dd, auto f) {
             return launch_nd_backward<decltype(dd)::value, decltype(f)::value, __half>(h, x, dL_dout, N, d, s);
@@ -621,6 +719,7 @@ int hashgrid_backward_half(hashgrid_t h, const float* x, const float* dL_dout, i
         case 8: return launch_backward_half<8>(h, x, dL_dout, N, d, s);
     }
     return fail(HASHGRID_ERR_ARG, "corrupt handle");
+    });
 }
 
 int hashgrid_backward_input(hashgrid_t h, const float* x, const float* dL_dout, int64_t N, const void* table,
@@ -634,6 +733,9 @@ int hashgrid_backward_input(hashgrid_t h, const float* x, const float* dL_dout, 
     if (int rc = check_buffer(table, table_bytes(h), "table")) return rc;
     if (int rc = check_buffer(dL_dx, (size_t)N * h->D * sizeof(float), "dL_dx")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    return run_checked(s, {{hg::kChkX, x, (size_t)N * h->D * sizeof(float)}, {hg::kChkDout, dL_dout, (size_t)N * W * sizeof(float)},
+                           {hg::kChkTable, table, table_bytes(h)}, {hg::kChkOut, dL_dx, (size_t)N * h->D * sizeof(float)}},
+                       "backward_input", [&]() -> int {
     const bool half = h->dtype == HASHGRID_F16;
     if (h->D != 3)
         return nd_dispatch(h, [&](auto d, auto f) {
@@ -648,6 +750,7 @@ int hashgrid_backward_input(hashgrid_t h, const float* x, const float* dL_dout, 
         case 8: return half ? launch_backward_input<8, __half>(h, x, dL_dout, N, table, dL_dx, s) : launch_backward_input<8, float>(h, x, dL_dout, N, table, dL_dx, s);
     }
     return fail(HASHGRID_ERR_ARG, "corrupt handle");
+    });
 }
 
 int hashgrid_adam_step(hashgrid_t h, void* table, float* adam_m, float* adam_v, float* dL_dtable, int64_t step,
@@ -677,11 +780,15 @@ int hashgrid_adam_step(hashgrid_t h, void* table, float* adam_m, float* adam_v, 
     const int64_t want = (n4 + 255) / 256;
     const unsigned blocks = (unsigned)(want < (int64_t)sms * 16 ? want : (int64_t)sms * 16);
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-    if (h->dtype == HASHGRID_F16)
-        hg::adam_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<__half*>(table), adam_m, adam_v, dL_dtable, n4, a, zero_grad);
-    else
-        hg::adam_kernel<float><<<blocks, 256, 0, s>>>(static_cast<float*>(table), adam_m, adam_v, dL_dtable, n4, a, zero_grad);
-    return launch_status("adam_step");
+    return run_checked(s, {{hg::kChkTable, table, table_bytes(h)}, {hg::kChkM, adam_m, n * sizeof(float)},
+                           {hg::kChkV, adam_v, n * sizeof(float)}, {hg::kChkGrad, dL_dtable, n * sizeof(float)}},
+                       "adam_step", [&]() -> int {
+        if (h->dtype == HASHGRID_F16)
+            hg::adam_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<__half*>(table), adam_m, adam_v, dL_dtable, n4, a, zero_grad);
+        else
+            hg::adam_kernel<float><<<blocks, 256, 0, s>>>(static_cast<float*>(table), adam_m, adam_v, dL_dtable, n4, a, zero_grad);
+        return launch_status("adam_step");
+    });
 }
 
 int hashgrid_mlp_forward(hashgrid_t h, const float* x, int64_t N, const void* table, const void* w1,
@@ -707,6 +814,9 @@ int hashgrid_mlp_forward(hashgrid_t h, const float* x, int64_t N, const void* ta
     if (device_status != nullptr)
         if (int rc = check_buffer(device_status, sizeof(int), "device_status")) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    return run_checked(s, {{hg::kChkX, x, (size_t)N * h->D * sizeof(float)}, {hg::kChkTable, table, table_bytes(h)},
+                           {hg::kChkOut, y, (size_t)N * kOut * sizeof(float)}},
+                       "mlp_forward", [&]() -> int {
     const bool half = h->dtype == HASHGRID_F16;
     switch (h->F) {
         case 1: return half ? dispatch_mlp_forward<1, __half>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, device_status, s)
@@ -719,6 +829,7 @@ int hashgrid_mlp_forward(hashgrid_t h, const float* x, int64_t N, const void* ta
                             : dispatch_mlp_forward<8, float>(h, x, N, table, w1, b1, w2, b2, w3, b3, y, device_status, s);
     }
     return fail(HASHGRID_ERR_ARG, "corrupt handle");
+    });
 }
 
 int hashgrid_debug_indices(hashgrid_t h, const float* x, int64_t N, uint32_t* idx_out, void* cuda_stream) {
@@ -732,13 +843,17 @@ int hashgrid_debug_indices(hashgrid_t h, const float* x, int64_t N, uint32_t* id
     const int64_t blocks = (total + threads - 1) / threads;
     if (blocks > 0x7fffffffLL) return fail(HASHGRID_ERR_ARG, "N too large for the index export");
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-    if (h->D == 2)
-        hg::nd::indices_kernel<2><<<(unsigned)blocks, threads, 0, s>>>(h->lp, x, N, idx_out);
-    else if (h->D == 4)
-        hg::nd::indices_kernel<4><<<(unsigned)blocks, threads, 0, s>>>(h->lp, x, N, idx_out);
-    else
-        hg::indices_kernel<<<(unsigned)blocks, threads, 0, s>>>(h->lp, x, N, idx_out);
-    return launch_status("debug_indices");
+    return run_checked(s, {{hg::kChkX, x, (size_t)N * h->D * sizeof(float)},
+                           {hg::kChkOut, idx_out, (size_t)N * h->L * ((size_t)1 << h->D) * sizeof(uint32_t)}},
+                       "debug_indices", [&]() -> int {
+        if (h->D == 2)
+            hg::nd::indices_kernel<2><<<(unsigned)blocks, threads, 0, s>>>(h->lp, x, N, idx_out);
+        else if (h->D == 4)
+            hg::nd::indices_kernel<4><<<(unsigned)blocks, threads, 0, s>>>(h->lp, x, N, idx_out);
+        else
+            hg::indices_kernel<<<(unsigned)blocks, threads, 0, s>>>(h->lp, x, N, idx_out);
+        return launch_status("debug_indices");
+    });
 }
 
 int hashgrid_probe(int kind, int width, int pattern, void* buf, size_t buf_bytes, int64_t ops, float* sink,

@@ -39,7 +39,11 @@ constexpr int kOutPad = 16;    // MMA N of the last layer (the smallest N for M 
 // Threads per CTA: 4 consumer warps + 20 producer warps (F <= 4, 40 registers a thread) or
 // + 12 (F = 8, 64 registers); 2 CTAs per SM either way. Two CTAs of 768 rather than three
 // of 512 gives more gathering warps per SM and leaves L1 more room beside shared memory.
-__host__ __device__ constexpr int block_threads(int F) { return F == 8 ? 512 : 768; }
+// With lane-pair producers (F <= 4): 4 + 16 warps, so that the 256 producer pairs cover
+// the 128 points of a tile exactly twice (48 registers a thread).
+__host__ __device__ constexpr int block_threads(int F, bool lanes = false) {
+    return lanes && F <= 4 ? 640 : (F == 8 ? 512 : 768);
+}
 constexpr int kCtasPerSm = 2;
 constexpr int kTmemCols = 64;  // accumulator columns (fp32), reused by the three layers
 constexpr uint32_t kWaitLimit = 1u << 22;
@@ -161,14 +165,15 @@ __device__ __forceinline__ bool consumers_any(bool pred) {
 // the current tile's MMAs and epilogues. Every wait is bounded: a consumer that gives up
 // makes all consumers stop together (the barrier vote) and raises the CTA's abort flag,
 // which stops the producers before their next tile; the caller's status word is then set.
-template <int F, typename TT, int K1>
-__global__ void __launch_bounds__(block_threads(F), kCtasPerSm) mlp_forward_kernel(
+template <int F, typename TT, int K1, bool kLanes = false>
+__global__ void __launch_bounds__(block_threads(F, kLanes), kCtasPerSm) mlp_forward_kernel(
     LevelParams lp, const float* __restrict__ x, int64_t N, const TT* __restrict__ table,
     const uint16_t* __restrict__ w1, const float* __restrict__ b1, const uint16_t* __restrict__ w2,
     const float* __restrict__ b2, const uint16_t* __restrict__ w3, const float* __restrict__ b3,
     float* __restrict__ y, int* __restrict__ status) {
     static_assert(K1 % 16 == 0 && K1 <= 64, "the encoding width must be a multiple of 16, at most 64");
-    constexpr int kThreads = block_threads(F);
+    static_assert(!kLanes || F <= 4, "lane-pair producers need F <= 4");
+    constexpr int kThreads = block_threads(F, kLanes);
     constexpr int kConsumers = kM;                     // 4 warps
     constexpr int kProducers = kThreads - kConsumers;  // 20 or 12 warps
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -221,10 +226,15 @@ __global__ void __launch_bounds__(block_threads(F), kCtasPerSm) mlp_forward_kern
         // x is read once per tile) and encodes every kStride-th level group of it; a warp
         // covers 32 consecutive points of one group. A group of G levels packs G*F bf16 values
         // into one 4-, 8- or 16-byte store within one core-matrix row.
-        static_assert(kProducers % kM == 0, "each producer thread owns one point of the tile");
+        // With kLanes, a lane pair (the two threads 2j, 2j+1) shares one point of one level
+        // group, thread d gathering the 4 corners with x offset d (as forward_kernel_lanes).
+        constexpr int kPer = kLanes ? 2 : 1;  // threads per (point, group)
+        static_assert(kProducers % (kM * kPer) == 0, "each producer thread (pair) owns one point of the tile");
         constexpr int G = F == 1 ? 2 : 1;
-        constexpr int kStride = kProducers / kM;
-        const int pt = tid - kConsumers, q = pt & (kM - 1), ngroups = lp.L / G;
+        constexpr int kStride = kProducers / (kM * kPer);
+        const int pt = (tid - kConsumers) / kPer, q = pt & (kM - 1), ngroups = lp.L / G;
+        const uint32_t d0 = (uint32_t)lane & 1u;
+        const unsigned pair = 3u << (lane & 30);
         for (int i = 0; i < my_tiles; ++i) {
             const int b = i & 1;
             bool stop = i >= 2 && !wait_parity(bar0 + 16 + 8 * b, (uint32_t)(((i >> 1) - 1) & 1));
@@ -235,8 +245,9 @@ __global__ void __launch_bounds__(block_threads(F), kCtasPerSm) mlp_forward_kern
             }
             const int64_t p = ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * kM + q;
             const bool valid = p < N;
-            const float x0 = valid ? __ldg(x + p * 3) : 0.f, x1 = valid ? __ldg(x + p * 3 + 1) : 0.f,
-                        x2 = valid ? __ldg(x + p * 3 + 2) : 0.f;
+            const bool xin = valid && in_bounds<kChkX>(x + p * 3, 12);
+            const float x0 = xin ? __ldg(x + p * 3) : 0.f, x1 = xin ? __ldg(x + p * 3 + 1) : 0.f,
+                        x2 = xin ? __ldg(x + p * 3 + 2) : 0.f;
             uint8_t* A0 = sm + b * (kM * K1 * 2);
             // The first group rotates with the tile, so that no warp always draws the extra
             // group when kStride does not divide the group count.
@@ -247,20 +258,30 @@ __global__ void __launch_bounds__(block_threads(F), kCtasPerSm) mlp_forward_kern
 #pragma unroll 1
                 for (int u = 0; u < G; ++u) {
                     const int l = gi * G + u;
-                    Corners cr;
-                    locate_corners(x0, x1, x2, lp.scale[l], lp.mask, cr);
-                    float e[8][F];
-                    gather_corners<F, TT, kGatherCorner, std::is_same<TT, float>::value>(table + (uint64_t)l * lp.T * F, cr, e);
+                    float acc[F];
+                    if constexpr (kLanes) {
+                        HalfCorners hc;
+                        locate_half(x0, x1, x2, lp.scale[l], lp.mask, d0, hc);
+                        interpolate_pair<F, TT>(table + (uint64_t)l * lp.T * F, hc, pair, acc);
+                    } else {
+                        Corners cr;
+                        locate_corners(x0, x1, x2, lp.scale[l], lp.mask, cr);
+                        float e[8][F];
+                        gather_corners<F, TT, kGatherCorner, std::is_same<TT, float>::value>(table + (uint64_t)l * lp.T * F, cr, e);
 #pragma unroll
-                    for (int f = 0; f < F; ++f) {
-                        float acc = cr.w[0] * e[0][f];
+                        for (int f = 0; f < F; ++f) {
+                            acc[f] = cr.w[0] * e[0][f];
 #pragma unroll
-                        for (int c = 1; c < 8; ++c) acc = fmaf(cr.w[c], e[c][f], acc);
+                            for (int c = 1; c < 8; ++c) acc[f] = fmaf(cr.w[c], e[c][f], acc[f]);
+                        }
+                    }
+#pragma unroll
+                    for (int f = 0; f < F; ++f)
 #pragma unroll
                         for (int uu = 0; uu < G; ++uu)  // constant indices: o stays in registers
-                            if (uu == u) o[uu * F + f] = acc;
-                    }
+                            if (uu == u) o[uu * F + f] = acc[f];
                 }
+                if (kLanes && d0 != 0) continue;  // both threads of a pair hold the sums; one stores
                 uint8_t* dst = A0 + canon(q, gi * G * F, K1);  // G*F consecutive columns, one 16-byte row chunk
                 if constexpr (G * F == 2) {
                     *reinterpret_cast<uint32_t*>(dst) = pack_bf16(o[0], o[1]);
@@ -329,7 +350,7 @@ __global__ void __launch_bounds__(block_threads(F), kCtasPerSm) mlp_forward_kern
                     float v[16];
                     tmem_ld16(trow, v);
                     const int64_t p = p0 + r;
-                    if (ok && p < N)
+                    if (ok && p < N && in_bounds<kChkOut>(y + p * kOut, 16))
                         __stcs(reinterpret_cast<float4*>(y + p * kOut),
                                make_float4(v[0] + bl[0], v[1] + bl[1], v[2] + bl[2], v[3] + bl[3]));
                 }

@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const floa
     float* os = smem + kTile * D;
     const int64_t p0 = (int64_t)blockIdx.x * kTile;
     const int nvalid = (int)min((int64_t)kTile, N - p0);
-    for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) xs[i] = __ldcs(x + p0 * D + i);
+    for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) xs[i] = ld_x(x + p0 * D + i);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     for (int it = warp; it < (kTile / 32) * L; it += nwarps) {
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
     float* gs = smem + kTile * D;
     const int64_t p0 = (int64_t)blockIdx.x * kTile;
     const int nvalid = (int)min((int64_t)kTile, N - p0);
-    for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) xs[i] = __ldcs(x + p0 * D + i);
+    for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) xs[i] = ld_x(x + p0 * D + i);
     stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(512) backward_input_kernel(LevelParams lp, con
     float* part = gs + kTile * S;  // [L][D][kTile]
     const int64_t p0 = (int64_t)blockIdx.x * kTile;
     const int nvalid = (int)min((int64_t)kTile, N - p0);
-    for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) xs[i] = __ldcs(x + p0 * D + i);
+    for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) xs[i] = ld_x(x + p0 * D + i);
     stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(512) backward_input_kernel(LevelParams lp, con
         const int pt = t / D, i = t - D * (t / D);
         float s = 0.f;
         for (int l = 0; l < L; ++l) s += part[(l * D + i) * kTile + pt];
-        __stcs(dx + p0 * D + t, s);
+        if (in_bounds<kChkOut>(dx + p0 * D + t, 4)) __stcs(dx + p0 * D + t, s);
     }
 }
 
@@ -194,11 +194,12 @@ __global__ void __launch_bounds__(256) indices_kernel(LevelParams lp, const floa
     const int l = (int)(t - p * lp.L);
     float xp[D];
 #pragma unroll
-    for (int i = 0; i < D; ++i) xp[i] = x[p * D + i];
+    for (int i = 0; i < D; ++i) xp[i] = ld_x(x + p * D + i);
     CornersND<D> cr;
     locate<D>(xp, lp.scale[l], lp.mask, cr);
 #pragma unroll
-    for (int c = 0; c < CornersND<D>::kC; ++c) idx[t * CornersND<D>::kC + c] = cr.idx[c];
+    for (int c = 0; c < CornersND<D>::kC; ++c)
+        if (in_bounds<kChkOut>(idx + t * CornersND<D>::kC + c, 4)) idx[t * CornersND<D>::kC + c] = cr.idx[c];
 }
 
 }  // namespace nd

@@ -472,7 +472,23 @@ def test_backward_input_widths_edges(F, dtype, gather):
     check_backward_x(og, x, table, g, got.cpu().numpy())
 
 
-@pytest.mark.parametrize("gather", ["auto", "lanes"])
+@pytest.mark.parametrize("gather", ["corner", "lanes"])
+@pytest.mark.parametrize("shape", [(32, 2, 12, 4, 4096), (32, 4, 10, 2, 300), (32, 8, 8, 2, 300), (1, 2, 10, 64, 64)])
+def test_backward_input_row_widths(shape, gather):
+    """Rows of 64 to 256 floats (the lane-pair kernel stages a warp's upstream-gradient rows
+    in shared memory, with fewer warps per block above 64 floats) and a single level."""
+    L, F, log2T, a, b = shape
+    grid, og = make_pair(L, F, log2T, a, b, gather=gather)
+    rng = np.random.default_rng(L * 10 + F)
+    table = workloads.table_values(rng, L, 2**log2T, F)
+    x = workloads.uniform_points(rng, 1000 + 13)
+    g = workloads.upstream_grads(rng, x.shape[0], L * F)
+    got = grid.backward_input(dev(x), dev(g), dev(table))
+    torch.cuda.synchronize()
+    check_backward_x(og, x, table, g, got.cpu().numpy())
+
+
+@pytest.mark.parametrize("gather", ["auto", "corner"])
 def test_backward_input_full_size_sampled(gather):
     """2^20 ray samples through the library's launch configuration; sampled rows checked."""
     w = workloads.WORKLOADS["rays_L16F2T19"]
@@ -621,10 +637,12 @@ def check_mlp(og, x, table, wts, got):
                                    (16, 1, 12, 16, 512, "f32"), (32, 1, 10, 8, 1000, "f16"),     # F = 1: two levels per store
                                    (4, 8, 12, 4, 200, "f32"), (8, 8, 12, 4, 300, "f16"),         # F = 8: 512-thread CTAs
                                    (12, 4, 12, 4, 300, "f16")])
-def test_mlp_forward_parity(shape):
+@pytest.mark.parametrize("gather", ["auto", "corner"])
+def test_mlp_forward_parity(shape, gather):
+    """Lane-pair producers (AUTO, F <= 4) and per-corner producers (CORNER, and F = 8)."""
     hg = hgmod()
     L, F, log2T, a, b, dtype = shape
-    grid, og = make_pair(L, F, log2T, a, b, dtype)
+    grid, og = make_pair(L, F, log2T, a, b, dtype, gather=gather)
     rng = np.random.default_rng(70 + L * F)
     table = (rng.standard_normal((L, 2**log2T, F)) * 0.3).astype(np.float32)
     if dtype == "f16":
@@ -656,14 +674,15 @@ def test_mlp_forward_full_size_sampled():
     check_mlp(og, inp.x[rows], table, wts, y.cpu().numpy()[rows])
 
 
+@pytest.mark.parametrize("gather", ["auto", "corner"])
 @pytest.mark.parametrize("N", [0, 1, 127, 128, 129, 3 * 2 * 148 * 128 + 77])
-def test_mlp_forward_tile_edges(N):
+def test_mlp_forward_tile_edges(N, gather):
     """Below, at and above one 128-point tile, and enough tiles that every persistent CTA
     cycles both encoding buffers at least once (3+ tiles per CTA): every row against the
     oracle; N = 0 writes nothing. Two calls give bit-identical results (no atomics)."""
     hg = hgmod()
     w = workloads.WORKLOADS["rays_L16F2T19"]
-    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max)
+    grid, og = make_pair(w.L, w.F, w.log2T, w.N_min, w.N_max, gather=gather)
     rng = np.random.default_rng(72)
     table = (rng.standard_normal((w.L, w.T, w.F)) * 0.3).astype(np.float32)
     x = workloads.ray_points(rng, (N + 63) // 64)[:N].astype(np.float32).reshape(-1, 3)
