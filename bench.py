@@ -540,6 +540,27 @@ def time_next_rows(res: Resident, steps: int, warmup: int, device, l2peaks=None)
                                    tensor_tflops=round(flops / (ms * 1e-3) / 1e12, 2))
         launches += steps
 
+    # D-dimensional inputs (D = 2, 4; 2^D corners, the 7-prime hash): forward and backward on
+    # N uniform points of the same grid.
+    nd = {}
+    for D in (2, 4):
+        gen = np.random.default_rng(1000 + D)
+        xd = torch.from_numpy(gen.random((N, D), dtype=np.float32)).to(device)
+        hd = hg.hashgrid_create_nd(D, w.L, w.F, w.log2T, w.N_min, w.N_max,
+                                   hg.HASHGRID_F16 if w.dtype == "f16" else hg.HASHGRID_F32)
+        outd = torch.empty((N, LF), dtype=torch.float32, device=device)
+        dtd = torch.zeros((w.L, w.T, w.F), dtype=torch.float32, device=device)
+        fms = time_launches(lambda: hg.hashgrid_forward(hd, xd, N, res.table, outd, sp), steps, warmup, device)
+        bms = time_launches(lambda: hg.hashgrid_backward(hd, xd, res.g, N, dtd, sp), steps, warmup, device,
+                            before=dtd.zero_)
+        hg.hashgrid_destroy(hd)
+        nd[f"D{D}"] = {"fwd_ms": round(fms, 5), "bwd_ms": round(bms, 5),
+                       "fwd_points_per_s": round(N / (fms * 1e-3), 1), "bwd_points_per_s": round(N / (bms * 1e-3), 1),
+                       "gathers_per_point": (1 << D) * w.L}
+        launches += 2 * steps
+        del xd, outd, dtd
+    out["nd"] = {"workload": f"{w.name} grid, {N} uniform points in [0,1)^D", **nd}
+
     # Backward into an fp16 gradient table (packed f16x2 reductions), zeroed before each call.
     dh = torch.zeros((w.L, w.T, w.F), dtype=torch.float16, device=device)
     ms = time_launches(lambda: hg.hashgrid_backward_half(res.handle, res.x, res.g, N, dh, sp), steps, warmup,

@@ -108,8 +108,11 @@ int hashgrid_create(int L, int F, int log2T, int N_min, int N_max, int dtype, ha
  * prod_i (offset_i ? frac_i : 1 - frac_i), corner c having offset bit i = (c >> i) & 1.
  * x is then [N, D] and dL_dx [N, D]; hashgrid_debug_indices writes [N, L, 2^D].
  * D = 3 is hashgrid_create. For D != 3 the forward pass gathers per corner and the backward
- * passes reduce per point (the gather, backward-mode and schedule options apply to D = 3
- * only), and hashgrid_mlp_forward is not available.
+ * passes reduce per point, with lane pairs (two threads per point and level, split by x
+ * offset) under the LANES gather option (forward, dL/dx) and the RUN_LANES backward option,
+ * and under AUTO for D = 4 (for D = 2 one thread per point and level measured faster); the
+ * schedule option and the other backward modes apply to D = 3 only, and
+ * hashgrid_mlp_forward is not available.
  */
 int hashgrid_create_nd(int D, int L, int F, int log2T, int N_min, int N_max, int dtype,
                        hashgrid_t *out);

@@ -1137,6 +1137,20 @@ template <> struct RedLane<2, __half> {
         asm volatile("red.global.add.noftz.f16x2 [%0], %1;" ::"l"(p), "r"(w) : "memory");
     }
 };
+template <> struct RedLane<8, __half> {
+    static __device__ __forceinline__ void add(__half* p, const float (&v)[8]) {
+        if (!in_bounds<kChkGrad>(p, 16)) return;
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            __half2 h = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
+            w[k] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        asm volatile("red.global.add.noftz.v4.f16x2 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                     "r"(w[3])
+                     : "memory");
+    }
+};
 template <> struct RedLane<4, __half> {
     static __device__ __forceinline__ void add(__half* p, const float (&v)[4]) {
         if (!in_bounds<kChkGrad>(p, 8)) return;

@@ -5,10 +5,10 @@
 // 805459861, 3674653429, 2097192037, 1434869437, 2165219737). A D-dimensional point
 // interpolates the 2^D corners of its cell with multilinear weights
 // prod_i (offset_i ? frac_i : 1 - frac_i); corner c has offset bit i = (c >> i) & 1.
-// These kernels follow the 3-D ones in hg_device.cuh (one thread per (point, level), a warp
-// = 32 consecutive points at one level, tiles of 64 points staged in shared memory, x-pair
-// merged reductions: the first prime is 1 here too), with per-corner gathers and per-point
-// reductions only.
+// These kernels follow the 3-D ones in hg_device.cuh (tiles of 64 points staged in shared
+// memory; by default lane pairs, two threads per (point, level) split by x offset, since the
+// first prime is 1 here too; otherwise one thread per (point, level) with x-pair merged
+// reductions), with per-corner gathers and per-point reductions only.
 #pragma once
 
 #include "hg_device.cuh"
@@ -56,13 +56,56 @@ __device__ __forceinline__ void locate(const float* xp, float scale, uint32_t ma
     }
 }
 
+// The 2^(D-1) corners with x offset d0 (lane d0 of a lane pair, as the 3-D lane-pair
+// kernels): corner k of the half is full corner c = d0 | (k << 1); index and weight as locate
+// computes them for that corner.
+template <int D>
+struct HalfCornersND {
+    static constexpr int kC = 1 << (D - 1);
+    uint32_t idx[kC];
+    float w[kC];
+    float f[D];
+};
+
+template <int D>
+__device__ __forceinline__ void locate_half(const float* xp, float scale, uint32_t mask, uint32_t d0,
+                                            HalfCornersND<D>& cr) {
+    uint32_t h0[D], h1[D];
+    float g[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+        const float xs = __fmul_rn(xp[i], scale);
+        const int v = __float2int_rd(xs);
+        cr.f[i] = __fsub_rn(xs, __int2float_rn(v));
+        g[i] = 1.0f - cr.f[i];
+        h0[i] = (uint32_t)v * kPrimes[i];
+        h1[i] = h0[i] + kPrimes[i];
+    }
+#pragma unroll
+    for (int k = 0; k < HalfCornersND<D>::kC; ++k) {
+        const int c = (int)d0 | (k << 1);
+        uint32_t h = 0;
+        float w = 1.0f;
+#pragma unroll
+        for (int i = 0; i < D; ++i) {
+            const bool b = (c >> i) & 1;
+            h ^= b ? h1[i] : h0[i];
+            w *= b ? cr.f[i] : g[i];
+        }
+        cr.idx[k] = h & mask;
+        cr.w[k] = w;
+    }
+}
+
 constexpr int kTile = 64;
 
 __host__ __device__ constexpr size_t tile_smem_bytes(int D, int L, int F) {
     return sizeof(float) * ((size_t)kTile * D + (size_t)kTile * (L * F + row_pad(F)));
 }
 
-template <int D, int F, typename TT>
+// kLanes: a warp item is 16 points at one level as 16 lane pairs, lane d handling the 2^(D-1)
+// corners with x offset d (the x prime is 1 here too); the pair adds its halves.
+template <int D, int F, typename TT, bool kLanes = false>
 __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const float* __restrict__ x, int64_t N,
                                                       const TT* __restrict__ table, float* __restrict__ out) {
     extern __shared__ __align__(16) float smem[];
@@ -74,6 +117,33 @@ __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const floa
     for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) xs[i] = ld_x(x + p0 * D + i);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    if constexpr (kLanes) {
+        const uint32_t d0 = lane & 1;
+        const unsigned pair = 3u << (lane & 30);
+        for (int it = warp; it < (kTile / 16) * L; it += nwarps) {
+            const int q = it / L, l = it - q * L, pl = q * 16 + (lane >> 1);
+            if (pl >= nvalid) continue;  // both lanes of a pair
+            HalfCornersND<D> cr;
+            locate_half<D>(xs + pl * D, lp.scale[l], lp.mask, d0, cr);
+            const TT* tl = table + (uint64_t)l * lp.T * F;
+            float o[F];
+#pragma unroll
+            for (int f = 0; f < F; ++f) o[f] = 0.f;
+#pragma unroll
+            for (int k = 0; k < HalfCornersND<D>::kC; ++k) {
+                float e[F];
+                EntryLoad<F, TT>::load(tl + (uint64_t)cr.idx[k] * F, e);
+#pragma unroll
+                for (int f = 0; f < F; ++f) o[f] = fmaf(cr.w[k], e[f], o[f]);
+            }
+#pragma unroll
+            for (int f = 0; f < F; ++f) o[f] += __shfl_xor_sync(pair, o[f], 1);
+            store_half<F, false>(os + pl * S + l * F, o, d0);
+        }
+        __syncthreads();
+        stage_rows_out<(F < 4 ? F : 4)>(os, out, p0, nvalid, W, S);
+        return;
+    }
     for (int it = warp; it < (kTile / 32) * L; it += nwarps) {
         const int q = it / L, l = it - q * L, pl = q * 32 + lane;
         if (pl >= nvalid) continue;
@@ -96,7 +166,9 @@ __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const floa
     stage_rows_out<(F < 4 ? F : 4)>(os, out, p0, nvalid, W, S);
 }
 
-template <int D, int F, typename GT>
+// kLanes: lane pairs as in the forward; each lane reduces its corners one F-wide reduction
+// each, so x-neighbouring corners are reduced by the same instruction.
+template <int D, int F, typename GT, bool kLanes = false>
 __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const float* __restrict__ x,
                                                        const float* __restrict__ dout, int64_t N, GT* __restrict__ dtable) {
     extern __shared__ __align__(16) float smem[];
@@ -109,6 +181,26 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
     stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    if constexpr (kLanes) {
+        const uint32_t d0 = lane & 1;
+        for (int it = warp; it < (kTile / 16) * L; it += nwarps) {
+            const int q = it / L, l = it - q * L, pl = q * 16 + (lane >> 1);
+            if (pl >= nvalid) continue;
+            HalfCornersND<D> cr;
+            locate_half<D>(xs + pl * D, lp.scale[l], lp.mask, d0, cr);
+            float g[F];
+            load_smem_entry<F>(gs + pl * S + l * F, g);
+            GT* dl = dtable + (uint64_t)l * lp.T * F;
+#pragma unroll
+            for (int k = 0; k < HalfCornersND<D>::kC; ++k) {
+                float v[F];
+#pragma unroll
+                for (int f = 0; f < F; ++f) v[f] = cr.w[k] * g[f];
+                RedLane<F, GT>::add(dl + (uint64_t)cr.idx[k] * F, v);
+            }
+        }
+        return;
+    }
     for (int it = warp; it < (kTile / 32) * L; it += nwarps) {
         const int q = it / L, l = it - q * L, pl = q * 32 + lane;
         if (pl >= nvalid) continue;
@@ -131,7 +223,8 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
 }
 
 // dL/dx_i = sum_l N_l sum_c (sum_f g e_c[f]) (d_i ? +1 : -1) prod_{j != i} (d_j ? frac_j : 1 - frac_j)
-template <int D, int F, typename TT>
+// kLanes: lane pairs as in the forward; the pair adds its halves of the D derivative sums.
+template <int D, int F, typename TT, bool kLanes = false>
 __global__ void __launch_bounds__(512) backward_input_kernel(LevelParams lp, const float* __restrict__ x,
                                                              const float* __restrict__ dout, int64_t N,
                                                              const TT* __restrict__ table, float* __restrict__ dx) {
@@ -146,6 +239,45 @@ __global__ void __launch_bounds__(512) backward_input_kernel(LevelParams lp, con
     stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    if constexpr (kLanes) {
+        const uint32_t d0 = lane & 1;
+        const unsigned pair = 3u << (lane & 30);
+        for (int it = warp; it < (kTile / 16) * L; it += nwarps) {
+            const int q = it / L, l = it - q * L, pl = q * 16 + (lane >> 1);
+            if (pl >= nvalid) continue;  // both lanes of a pair
+            HalfCornersND<D> cr;
+            locate_half<D>(xs + pl * D, lp.scale[l], lp.mask, d0, cr);
+            float g[F];
+            load_smem_entry<F>(gs + pl * S + l * F, g);
+            const TT* tl = table + (uint64_t)l * lp.T * F;
+            float d[D];
+#pragma unroll
+            for (int i = 0; i < D; ++i) d[i] = 0.f;
+#pragma unroll
+            for (int k = 0; k < HalfCornersND<D>::kC; ++k) {
+                const int c = (int)d0 | (k << 1);
+                float e[F];
+                EntryLoad<F, TT>::load(tl + (uint64_t)cr.idx[k] * F, e);
+                float sc = g[0] * e[0];
+#pragma unroll
+                for (int f = 1; f < F; ++f) sc = fmaf(g[f], e[f], sc);
+#pragma unroll
+                for (int i = 0; i < D; ++i) {
+                    float pw = ((c >> i) & 1) ? sc : -sc;
+#pragma unroll
+                    for (int j = 0; j < D; ++j)
+                        if (j != i) pw *= ((c >> j) & 1) ? cr.f[j] : 1.0f - cr.f[j];
+                    d[i] += pw;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < D; ++i) d[i] += __shfl_xor_sync(pair, d[i], 1);
+            if (d0 == 0) {
+#pragma unroll
+                for (int i = 0; i < D; ++i) part[(l * D + i) * kTile + pl] = lp.scale[l] * d[i];
+            }
+        }
+    } else {
     for (int it = warp; it < (kTile / 32) * L; it += nwarps) {
         const int q = it / L, l = it - q * L, pl = q * 32 + lane;
         if (pl >= nvalid) continue;
@@ -175,6 +307,7 @@ __global__ void __launch_bounds__(512) backward_input_kernel(LevelParams lp, con
         }
 #pragma unroll
         for (int i = 0; i < D; ++i) part[(l * D + i) * kTile + pl] = lp.scale[l] * d[i];
+    }
     }
     __syncthreads();
     for (int t = threadIdx.x; t < nvalid * D; t += blockDim.x) {

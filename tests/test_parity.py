@@ -792,15 +792,24 @@ def test_backward_half_widths(F, mode):
 # D-dimensional inputs
 # ---------------------------------------------------------------------------------------
 
+ND_MODES = {"auto": {}, "lanes": {"forward_gather": 4, "backward_mode": 5},           # LANES, RUN_LANES
+            "one-lane": {"forward_gather": 1, "backward_mode": 1}}                      # CORNER, ATOMIC
+
+
+@pytest.mark.parametrize("mode", list(ND_MODES))
 @pytest.mark.parametrize("F", [1, 2, 4, 8])
 @pytest.mark.parametrize("D", [2, 4])
-def test_nd_parity(D, F):
+def test_nd_parity(D, F, mode):
     """Indices bit-exact, forward within 1e-6 of sum_c w_c |e_c| (2^D products of D-1
     fp32 roundings and 2^D fma: ~(D + 2^D) ulp), fp32 and fp16 gradients, and dL/dx, for
-    D = 2 and 4 against the oracle's D-dimensional functions."""
+    D = 2 and 4 against the oracle's D-dimensional functions; lane-pair kernels (LANES,
+    RUN_LANES), one thread per (point, level) (CORNER gathers, ATOMIC reductions) and AUTO."""
     hg = hgmod()
     L, log2T = 6, 12
-    grid = hg.HashGrid(L, F, log2T, 3, 150, D=D)
+    opts = dict(ND_MODES[mode])
+    if F > 4 and opts.get("backward_mode") == 5:   # RUN_LANES takes F <= 4 (AUTO covers D = 4, F = 8 lanes)
+        opts["backward_mode"] = 1
+    grid = hg.HashGrid(L, F, log2T, 3, 150, D=D, **opts)
     og = oracle.GridND(D, L, F, log2T, 3, 150)
     rng = np.random.default_rng(100 + 10 * D + F)
     table = workloads.table_values(rng, L, 2**log2T, F)
@@ -829,14 +838,15 @@ def test_nd_parity(D, F):
     assert np.all(np.abs(dx - dxref) <= 1e-5 * B[:, None] * 2 ** (D - 3) + 1e-30)
 
 
+@pytest.mark.parametrize("mode", list(ND_MODES))
 @pytest.mark.parametrize("F", [2, 4])
 @pytest.mark.parametrize("D", [2, 4])
-def test_nd_parity_fp16_table(D, F):
+def test_nd_parity_fp16_table(D, F, mode):
     """fp16 tables with D = 2 and 4: the entries are decoded exactly, so the forward holds
     the fp32 bound (1e-6 of sum_c w_c |e_c|) and dL/dx the same bound as with fp32 tables."""
     hg = hgmod()
     L, log2T = 6, 12
-    grid = hg.HashGrid(L, F, log2T, 3, 150, dtype=hg.HASHGRID_F16, D=D)
+    grid = hg.HashGrid(L, F, log2T, 3, 150, dtype=hg.HASHGRID_F16, D=D, **ND_MODES[mode])
     og = oracle.GridND(D, L, F, log2T, 3, 150, dtype=oracle.F16)
     rng = np.random.default_rng(120 + 10 * D + F)
     table = (rng.standard_normal((L, 2**log2T, F)) * 0.5).astype(np.float16)
