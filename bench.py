@@ -2,20 +2,25 @@
 """Benchmark of the multiresolution hash-grid encoding on B200: encoded points/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload NAME] [--skip-cpu-baseline] [--skip-e2e] [--skip-fwd-leg]
-                    [--skip-next-rows]
+                    [--workload NAME] [--points N] [--min-timed-s S] [--skip-cpu-baseline]
+                    [--skip-e2e] [--skip-legs] [--skip-peaks] [--skip-next-rows]
 
 One step = one pass of the whole hot path over one batch resident in HBM: forward (voxel,
 8 corner hashes, gathers, trilinear interpolation, level-major output rows), zero the table
 gradient, backward (weighted scatter-add into the fp32 gradient table). The default
 workload is the 16-level, F=2, T=2^19 grid (N 16->512) on 2^14 rays x 64 stratified
-samples (2^20 points); the forward-only leg on 2^18 uniform points of the same grid is
-reported under "fwd", and the gradient w.r.t. x, a sparse Adam step, the encoding fused with
-the MLP and the fp16-gradient backward on the same batch under "next_rows". L2 is flushed
-(256 MiB write) before every timed step, outside the step's events. Rank 0 prints one JSON
-line.
+samples (2^20 points). W warm-up steps, then the K-step loop runs R times back to back so
+that the timed region lasts at least --min-timed-s (all R*K steps timed with CUDA events,
+L2 flushed by a 256 MiB write before every step, outside its events). Rank 0 prints one
+JSON line with the rate, per-kernel rooflines (HBM basis, and the L2 basis against the
+gather / reduction rates the probe kernels measure in the same run), clocks, the other
+workloads as "legs" (forward-only grid on 2^18 uniform points, also under "fwd"; fp16
+table; 1 GiB grid), "next_rows" (dL/dx, sparse Adam, encoding + MLP, 2-D / 4-D inputs,
+fp16-gradient backward), an end-to-end figure through the C ABI from pinned host memory,
+and the CPU oracle's rate.
 
-Multi-GPU: one process per GPU (torchrun); every rank encodes its own batch with its own
+Multi-GPU: one process per GPU (``--gpus N`` starts the N ranks through
+torch.distributed.run when no launcher did); every rank encodes its own batch with its own
 table replica (points are independent), there is no collective on the data path, and the
 value is all ranks' points divided by the slowest rank's time (weak scaling).
 
@@ -587,7 +592,7 @@ def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, ke
     HBM (the primary fraction, bound "hbm"): the algorithmic bytes of the launch (x, the
     table gathers or fp32 reductions counted once each, the output or upstream-gradient
     rows) at the measured HBM copy bandwidth.
-    L2 (the benchmark spec: the gather roofline is L2 for tables that fit in it): the 8 * L table
+    L2 (the gather roofline of a table that fits in L2 is L2's, not HBM's): the 8 * L table
     gathers (fwd) or corner reductions (bwd) per point at the rate this device serves the
     hash's access pattern from an L2-resident buffer of the working set's size: x-neighbour
     pairs of F*s-byte entries (fwd) or F-wide fp32 / fp16 contributions (bwd), measured in
