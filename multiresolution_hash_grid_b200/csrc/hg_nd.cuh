@@ -140,27 +140,25 @@ __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const floa
             for (int f = 0; f < F; ++f) o[f] += __shfl_xor_sync(pair, o[f], 1);
             store_half<F, false>(os + pl * S + l * F, o, d0);
         }
-        __syncthreads();
-        stage_rows_out<(F < 4 ? F : 4)>(os, out, p0, nvalid, W, S);
-        return;
-    }
-    for (int it = warp; it < (kTile / 32) * L; it += nwarps) {
-        const int q = it / L, l = it - q * L, pl = q * 32 + lane;
-        if (pl >= nvalid) continue;
-        CornersND<D> cr;
-        locate<D>(xs + pl * D, lp.scale[l], lp.mask, cr);
-        const TT* tl = table + (uint64_t)l * lp.T * F;
-        float o[F];
+    } else {
+        for (int it = warp; it < (kTile / 32) * L; it += nwarps) {
+            const int q = it / L, l = it - q * L, pl = q * 32 + lane;
+            if (pl >= nvalid) continue;
+            CornersND<D> cr;
+            locate<D>(xs + pl * D, lp.scale[l], lp.mask, cr);
+            const TT* tl = table + (uint64_t)l * lp.T * F;
+            float o[F];
 #pragma unroll
-        for (int f = 0; f < F; ++f) o[f] = 0.f;
+            for (int f = 0; f < F; ++f) o[f] = 0.f;
 #pragma unroll
-        for (int c = 0; c < CornersND<D>::kC; ++c) {
-            float e[F];
-            EntryLoad<F, TT>::load(tl + (uint64_t)cr.idx[c] * F, e);
+            for (int c = 0; c < CornersND<D>::kC; ++c) {
+                float e[F];
+                EntryLoad<F, TT>::load(tl + (uint64_t)cr.idx[c] * F, e);
 #pragma unroll
-            for (int f = 0; f < F; ++f) o[f] = fmaf(cr.w[c], e[f], o[f]);
+                for (int f = 0; f < F; ++f) o[f] = fmaf(cr.w[c], e[f], o[f]);
+            }
+            store_smem_entry<F>(os + pl * S + l * F, o);
         }
-        store_smem_entry<F>(os + pl * S + l * F, o);
     }
     __syncthreads();
     stage_rows_out<(F < 4 ? F : 4)>(os, out, p0, nvalid, W, S);
@@ -199,25 +197,25 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
                 RedLane<F, GT>::add(dl + (uint64_t)cr.idx[k] * F, v);
             }
         }
-        return;
-    }
-    for (int it = warp; it < (kTile / 32) * L; it += nwarps) {
-        const int q = it / L, l = it - q * L, pl = q * 32 + lane;
-        if (pl >= nvalid) continue;
-        CornersND<D> cr;
-        locate<D>(xs + pl * D, lp.scale[l], lp.mask, cr);
-        float g[F];
-        load_smem_entry<F>(gs + pl * S + l * F, g);
-        GT* dl = dtable + (uint64_t)l * lp.T * F;
+    } else {
+        for (int it = warp; it < (kTile / 32) * L; it += nwarps) {
+            const int q = it / L, l = it - q * L, pl = q * 32 + lane;
+            if (pl >= nvalid) continue;
+            CornersND<D> cr;
+            locate<D>(xs + pl * D, lp.scale[l], lp.mask, cr);
+            float g[F];
+            load_smem_entry<F>(gs + pl * S + l * F, g);
+            GT* dl = dtable + (uint64_t)l * lp.T * F;
 #pragma unroll
-        for (int c = 0; c < CornersND<D>::kC; c += 2) {
-            float va[F], vb[F];
+            for (int c = 0; c < CornersND<D>::kC; c += 2) {
+                float va[F], vb[F];
 #pragma unroll
-            for (int f = 0; f < F; ++f) {
-                va[f] = cr.w[c] * g[f];
-                vb[f] = cr.w[c + 1] * g[f];
+                for (int f = 0; f < F; ++f) {
+                    va[f] = cr.w[c] * g[f];
+                    vb[f] = cr.w[c + 1] * g[f];
+                }
+                red_pair<F>(dl, cr.idx[c], cr.idx[c + 1], va, vb);
             }
-            red_pair<F>(dl, cr.idx[c], cr.idx[c + 1], va, vb);
         }
     }
 }
