@@ -602,7 +602,11 @@ def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, ke
     (all of them for a table larger than L2, else the x / output / upstream-gradient
     rows); frac_bound_time = bound_time / kernel time. Batches more coherent than the
     probe's independent random pairs (samples along rays share cache lines and voxels)
-    can exceed 1 on the L2 basis."""
+    can exceed 1 on the L2 basis. For the backward, the L2 reduction requests of the
+    launch (counted once by ncu for the committed kernel sources) are also set against the
+    rate at which the L2 serves independent random reductions of the same width, one
+    request each: the request-rate ceiling that merging x-neighbours or run-walk faces
+    does not move."""
     hbm, src = measured_peaks()
     s = 2 if w.dtype == "f16" else 4
     alg = algorithmic_bytes_per_point(w, kind) * points
@@ -640,7 +644,14 @@ def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, ke
     ent = ncu_entry(kernel, w.name)
     if ent is not None and ent.get("l2_red_requests_per_launch"):
         reds = float(ent["l2_red_requests_per_launch"])
-        out["l2_red_requests"] = {"per_launch": int(reds), "g_per_s": round(reds / (kernel_ms * 1e-3) / 1e9, 1)}
+        g_per_s = reds / (kernel_ms * 1e-3) / 1e9
+        out["l2_red_requests"] = {"per_launch": int(reds), "g_per_s": round(g_per_s, 1)}
+        if "l2" in out:
+            # one L2 request per operation when the units are independent and random
+            peak = rates["random"]
+            out["l2_red_requests"].update({"peak_g_per_s": peak, "frac": round(g_per_s / peak, 4),
+                                           "peak_source": f"hashgrid_probe, random {width}-byte units on a "
+                                                          f"{bkey} L2-resident buffer (one request each), this run"})
     return out
 
 

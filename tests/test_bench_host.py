@@ -52,6 +52,20 @@ def test_roofline_l2_basis(monkeypatch):
     assert h["algorithmic_bytes_per_launch"] == (12 + 128 + 8 * 32 * 2) * (1 << 20)
 
 
+def test_roofline_reduction_requests(monkeypatch):
+    """The backward's L2 reduction requests (an ncu count) against the random-unit
+    reduction rate of the same width: one request per operation."""
+    monkeypatch.setattr(bench, "measured_peaks", lambda: (5000.0, "test"))
+    monkeypatch.setattr(bench, "ncu_entry", lambda k, w: {"l2_red_requests_per_launch": 55e6, "dram_bytes_per_launch": 1e8})
+    b = bench.roofline(W["rays_L16F2T19"], "bwd", 1 << 20, 0.35, "backward_kernel", fake_peaks())
+    rr = b["l2_red_requests"]
+    assert rr["per_launch"] == 55_000_000 and rr["g_per_s"] == pytest.approx(55e6 / 0.35e-3 / 1e9, abs=0.05)
+    assert rr["peak_g_per_s"] == 100.0 and rr["frac"] == pytest.approx(55e6 / 0.35e-3 / 100e9, rel=1e-3)
+    assert "random 8-byte" in rr["peak_source"]
+    # without probe peaks only the count and rate are reported
+    assert "frac" not in bench.roofline(W["rays_L16F2T19"], "bwd", 1 << 20, 0.35, "backward_kernel", None)["l2_red_requests"]
+
+
 def test_roofline_large_grid_is_hbm_bound_per_level(monkeypatch):
     """The 1 GiB table does not fit in L2: every algorithmic byte crosses HBM, and the L2
     term uses one level's 64 MB slice (the level-major schedule's working set)."""
