@@ -180,35 +180,65 @@ __device__ __forceinline__ void sector_entry(const uint32_t (&w)[8], uint32_t j,
     }
 }
 
+// L2 policy that keeps lines resident (evict-last): the level-major kernels give it to the
+// gathers from, and the reductions into, the level's table or gradient slice, so that the
+// streamed rows (x, output, upstream gradient) do not push the slice out of L2.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 // ---------------------------------------------------------------------------------------
 // fp32 vector reductions into global memory (red.global.add, vector forms are sm_90+).
+// kKeep adds the evict-last L2 policy (the level-major backward: a 64 MB gradient slice
+// next to the streamed rows measured 2.91 ms with it and 3.41 ms without on the 1 GiB
+// grid; on L2-resident gradients it changes nothing).
 // ---------------------------------------------------------------------------------------
-template <int F> struct RedAdd;
-template <> struct RedAdd<1> {
+template <int F, bool kKeep = false> struct RedAdd;
+template <bool kKeep> struct RedAdd<1, kKeep> {
     static __device__ __forceinline__ void add(float* p, const float* v) {
         if (!in_bounds<kChkGrad>(p, 4)) return;
-        asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v[0]) : "memory");
+        if constexpr (kKeep) {
+            asm volatile("red.global.add.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v[0]),
+                         "l"(l2_evict_last_policy())
+                         : "memory");
+        } else {
+            asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v[0]) : "memory");
+        }
     }
 };
-template <> struct RedAdd<2> {
+template <bool kKeep> struct RedAdd<2, kKeep> {
     static __device__ __forceinline__ void add(float* p, const float* v) {
         if (!in_bounds<kChkGrad>(p, 8)) return;
-        asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(v[0]), "f"(v[1])
-                     : "memory");
+        if constexpr (kKeep) {
+            asm volatile("red.global.add.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(v[0]), "f"(v[1]),
+                         "l"(l2_evict_last_policy())
+                         : "memory");
+        } else {
+            asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(v[0]), "f"(v[1])
+                         : "memory");
+        }
     }
 };
-template <> struct RedAdd<4> {
+template <bool kKeep> struct RedAdd<4, kKeep> {
     static __device__ __forceinline__ void add(float* p, const float* v) {
         if (!in_bounds<kChkGrad>(p, 16)) return;
-        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v[0]),
-                     "f"(v[1]), "f"(v[2]), "f"(v[3])
-                     : "memory");
+        if constexpr (kKeep) {
+            asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v[0]),
+                         "f"(v[1]), "f"(v[2]), "f"(v[3]), "l"(l2_evict_last_policy())
+                         : "memory");
+        } else {
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v[0]),
+                         "f"(v[1]), "f"(v[2]), "f"(v[3])
+                         : "memory");
+        }
     }
 };
-template <> struct RedAdd<8> {
+template <bool kKeep> struct RedAdd<8, kKeep> {
     static __device__ __forceinline__ void add(float* p, const float* v) {
-        RedAdd<4>::add(p, v);
-        RedAdd<4>::add(p + 4, v + 4);
+        RedAdd<4, kKeep>::add(p, v);
+        RedAdd<4, kKeep>::add(p + 4, v + 4);
     }
 };
 
@@ -231,7 +261,7 @@ __device__ __forceinline__ void unit_vals(uint32_t i, const float* v, float (&u)
     }
 }
 
-template <int F>
+template <int F, bool kKeep = false>
 __device__ __forceinline__ void red_pair(float* dl, uint32_t a, uint32_t b, const float* va,
                                          const float* vb, bool ra = true, bool rb = true) {
     if constexpr (F <= 2) {
@@ -245,19 +275,20 @@ __device__ __forceinline__ void red_pair(float* dl, uint32_t a, uint32_t b, cons
 #pragma unroll
         for (int k = 0; k < 4; ++k) u1[k] = shared ? ua[k] + ub[k] : (ra ? ua[k] : ub[k]);
         const uint32_t i1 = ra ? a : b;
-        if (ra || rb) RedAdd<4>::add(dl + (uint64_t)(i1 & ~(kUnit - 1)) * F, u1);
+        if (ra || rb) RedAdd<4, kKeep>::add(dl + (uint64_t)(i1 & ~(kUnit - 1)) * F, u1);
         // second instruction: b's own unit when both are reduced but do not share one
-        if (ra && rb && !shared) RedAdd<4>::add(dl + (uint64_t)(b & ~(kUnit - 1)) * F, ub);
+        if (ra && rb && !shared) RedAdd<4, kKeep>::add(dl + (uint64_t)(b & ~(kUnit - 1)) * F, ub);
     } else {
-        if (ra) RedAdd<F>::add(dl + (uint64_t)a * F, va);
-        if (rb) RedAdd<F>::add(dl + (uint64_t)b * F, vb);
+        if (ra) RedAdd<F, kKeep>::add(dl + (uint64_t)a * F, va);
+        if (rb) RedAdd<F, kKeep>::add(dl + (uint64_t)b * F, vb);
     }
 }
 
 // fp16 gradient tables: 16-byte red.global.add.noftz.v4.f16x2 (sm_90+) on aligned units of
 // 8 halves (8 / F entries). Contributions are rounded to fp16 (round to nearest, subnormals
 // kept) and the L2 adds in fp16. Two x-corners share a unit more often than in fp32
-// (F = 2: when v0 mod 4 != 3), so fewer reductions reach L2.
+// (F = 2: when v0 mod 4 != 3), so fewer reductions reach L2. kKeep: evict-last, as RedAdd.
+template <bool kKeep = false>
 __device__ __forceinline__ void red_half_unit(__half* p, const float (&u)[8]) {
     if (!in_bounds<kChkGrad>(p, 16)) return;
     uint32_t w[4];
@@ -266,9 +297,15 @@ __device__ __forceinline__ void red_half_unit(__half* p, const float (&u)[8]) {
         __half2 h = __floats2half2_rn(u[2 * k], u[2 * k + 1]);
         w[k] = *reinterpret_cast<uint32_t*>(&h);
     }
-    asm volatile("red.global.add.noftz.v4.f16x2 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-                 "r"(w[3])
-                 : "memory");
+    if constexpr (kKeep) {
+        asm volatile("red.global.add.L2::cache_hint.noftz.v4.f16x2 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(w[0]),
+                     "r"(w[1]), "r"(w[2]), "r"(w[3]), "l"(l2_evict_last_policy())
+                     : "memory");
+    } else {
+        asm volatile("red.global.add.noftz.v4.f16x2 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                     "r"(w[3])
+                     : "memory");
+    }
 }
 
 template <int F>
@@ -284,7 +321,7 @@ __device__ __forceinline__ void unit_vals_half(uint32_t i, const float* v, float
     }
 }
 
-template <int F>
+template <int F, bool kKeep = false>
 __device__ __forceinline__ void red_pair(__half* dl, uint32_t a, uint32_t b, const float* va, const float* vb,
                                          bool ra = true, bool rb = true) {
     constexpr uint32_t kUnit = 8 / F;
@@ -295,8 +332,8 @@ __device__ __forceinline__ void red_pair(__half* dl, uint32_t a, uint32_t b, con
 #pragma unroll
     for (int k = 0; k < 8; ++k) u1[k] = shared ? ua[k] + ub[k] : (ra ? ua[k] : ub[k]);
     const uint32_t i1 = ra ? a : b;
-    if (ra || rb) red_half_unit(dl + (uint64_t)(i1 & ~(kUnit - 1)) * F, u1);
-    if (ra && rb && !shared) red_half_unit(dl + (uint64_t)(b & ~(kUnit - 1)) * F, ub);
+    if (ra || rb) red_half_unit<kKeep>(dl + (uint64_t)(i1 & ~(kUnit - 1)) * F, u1);
+    if (ra && rb && !shared) red_half_unit<kKeep>(dl + (uint64_t)(b & ~(kUnit - 1)) * F, ub);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -982,7 +1019,7 @@ __host__ __device__ constexpr size_t run_smem_bytes(int L, int F) {
     return sizeof(float) * ((size_t)32 * run_x_stride() + (size_t)32 * run_g_stride(L, F));
 }
 
-template <int F, typename GT>
+template <int F, bool kKeep = false, typename GT>
 __device__ __forceinline__ void run_flush(GT* dl, const float (&acc)[8][F], const uint32_t (&cidx)[8],
                                           int ax, uint32_t leave_bit) {
 #pragma unroll
@@ -990,14 +1027,14 @@ __device__ __forceinline__ void run_flush(GT* dl, const float (&acc)[8][F], cons
         const int a = 2 * q, b = 2 * q + 1;
         const bool fa = ax < 0 || (((uint32_t)a >> ax) & 1u) == leave_bit;
         const bool fb = ax < 0 || (((uint32_t)b >> ax) & 1u) == leave_bit;
-        red_pair<F>(dl, cidx[a], cidx[b], acc[a], acc[b], fa, fb);
+        red_pair<F, kKeep>(dl, cidx[a], cidx[b], acc[a], acc[b], fa, fb);
     }
 }
 
 // Walk one run of `n` consecutive points at one level (scale, mask) and reduce into the
 // level table dl. xp(j, x3) loads point j's 3 coordinates; gl(j, g) its F upstream
 // gradients.
-template <int F, typename GT, class XP, class GL>
+template <int F, bool kKeep = false, typename GT, class XP, class GL>
 __device__ __forceinline__ void walk_run(GT* dl, float scale, uint32_t mask, int n, XP xp, GL gl) {
     float acc[8][F];
     uint32_t cidx[8];
@@ -1019,7 +1056,7 @@ __device__ __forceinline__ void walk_run(GT* dl, float scale, uint32_t mask, int
                 const bool face = abs(dx) + abs(dy) + abs(dz) == 1;
                 const int ax = face ? (dx != 0 ? 0 : (dy != 0 ? 1 : 2)) : -1;
                 const uint32_t leave_bit = (dx + dy + dz) > 0 ? 0u : 1u;
-                run_flush<F>(dl, acc, cidx, ax, leave_bit);
+                run_flush<F, kKeep>(dl, acc, cidx, ax, leave_bit);
                 // carried corners: the new corner c with bit ax == leave_bit is the old
                 // corner c ^ (1 << ax); every other new corner starts from zero
                 float old[8][F];
@@ -1048,7 +1085,7 @@ __device__ __forceinline__ void walk_run(GT* dl, float scale, uint32_t mask, int
         cv1 = cr.v[1];
         cv2 = cr.v[2];
     }
-    if (n > 0) run_flush<F>(dl, acc, cidx, -1, 0u);
+    if (n > 0) run_flush<F, kKeep>(dl, acc, cidx, -1, 0u);
 }
 
 template <int F, typename GT>
@@ -1118,45 +1155,52 @@ __global__ void __launch_bounds__(256) backward_kernel_runs(LevelParams lp, cons
 // hands the shared face's 4 sums from one lane to the other with shuffles; y and z steps
 // carry sums inside each lane, as in walk_run.
 // ---------------------------------------------------------------------------------------
-template <int F, typename GT> struct RedLane;
-template <int F> struct RedLane<F, float> {
-    static __device__ __forceinline__ void add(float* p, const float (&v)[F]) { RedAdd<F>::add(p, v); }
+template <int F, typename GT, bool kKeep = false> struct RedLane;
+template <int F, bool kKeep> struct RedLane<F, float, kKeep> {
+    static __device__ __forceinline__ void add(float* p, const float (&v)[F]) { RedAdd<F, kKeep>::add(p, v); }
 };
-template <> struct RedLane<1, __half> {
+template <bool kKeep> struct RedLane<1, __half, kKeep> {
     static __device__ __forceinline__ void add(__half* p, const float (&v)[1]) {
         if (!in_bounds<kChkGrad>(p, 2)) return;
         const unsigned short h = __half_as_ushort(__float2half_rn(v[0]));
-        asm volatile("red.global.add.noftz.f16 [%0], %1;" ::"l"(p), "h"(h) : "memory");
+        if constexpr (kKeep) {
+            asm volatile("red.global.add.L2::cache_hint.noftz.f16 [%0], %1, %2;" ::"l"(p), "h"(h),
+                         "l"(l2_evict_last_policy())
+                         : "memory");
+        } else {
+            asm volatile("red.global.add.noftz.f16 [%0], %1;" ::"l"(p), "h"(h) : "memory");
+        }
     }
 };
-template <> struct RedLane<2, __half> {
+template <bool kKeep> struct RedLane<2, __half, kKeep> {
     static __device__ __forceinline__ void add(__half* p, const float (&v)[2]) {
         if (!in_bounds<kChkGrad>(p, 4)) return;
         __half2 h = __floats2half2_rn(v[0], v[1]);
         const uint32_t w = *reinterpret_cast<uint32_t*>(&h);
-        asm volatile("red.global.add.noftz.f16x2 [%0], %1;" ::"l"(p), "r"(w) : "memory");
-    }
-};
-template <> struct RedLane<8, __half> {
-    static __device__ __forceinline__ void add(__half* p, const float (&v)[8]) {
-        if (!in_bounds<kChkGrad>(p, 16)) return;
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            __half2 h = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
-            w[k] = *reinterpret_cast<uint32_t*>(&h);
+        if constexpr (kKeep) {
+            asm volatile("red.global.add.L2::cache_hint.noftz.f16x2 [%0], %1, %2;" ::"l"(p), "r"(w),
+                         "l"(l2_evict_last_policy())
+                         : "memory");
+        } else {
+            asm volatile("red.global.add.noftz.f16x2 [%0], %1;" ::"l"(p), "r"(w) : "memory");
         }
-        asm volatile("red.global.add.noftz.v4.f16x2 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-                     "r"(w[3])
-                     : "memory");
     }
 };
-template <> struct RedLane<4, __half> {
+template <bool kKeep> struct RedLane<8, __half, kKeep> {
+    static __device__ __forceinline__ void add(__half* p, const float (&v)[8]) { red_half_unit<kKeep>(p, v); }
+};
+template <bool kKeep> struct RedLane<4, __half, kKeep> {
     static __device__ __forceinline__ void add(__half* p, const float (&v)[4]) {
         if (!in_bounds<kChkGrad>(p, 8)) return;
         __half2 a = __floats2half2_rn(v[0], v[1]), b = __floats2half2_rn(v[2], v[3]);
         const uint32_t wa = *reinterpret_cast<uint32_t*>(&a), wb = *reinterpret_cast<uint32_t*>(&b);
-        asm volatile("red.global.add.noftz.v2.f16x2 [%0], {%1, %2};" ::"l"(p), "r"(wa), "r"(wb) : "memory");
+        if constexpr (kKeep) {
+            asm volatile("red.global.add.L2::cache_hint.noftz.v2.f16x2 [%0], {%1, %2}, %3;" ::"l"(p), "r"(wa),
+                         "r"(wb), "l"(l2_evict_last_policy())
+                         : "memory");
+        } else {
+            asm volatile("red.global.add.noftz.v2.f16x2 [%0], {%1, %2};" ::"l"(p), "r"(wa), "r"(wb) : "memory");
+        }
     }
 };
 
@@ -1169,7 +1213,7 @@ __device__ __forceinline__ void locate_half_voxel(float x0, float x1, float x2, 
     v[2] = __float2int_rd(__fmul_rn(x2, scale));
 }
 
-template <int F, typename GT, class XP, class GL>
+template <int F, bool kKeep = false, typename GT, class XP, class GL>
 __device__ __forceinline__ void walk_run_pair(GT* dl, float scale, uint32_t mask, int n, uint32_t d0, unsigned pair,
                                               XP xp, GL gl) {
     float acc[4][F];
@@ -1198,7 +1242,7 @@ __device__ __forceinline__ void walk_run_pair(GT* dl, float scale, uint32_t mask
                     const uint32_t leave = dx > 0 ? 0u : 1u;
                     if (d0 == leave) {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) RedLane<F, GT>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
+                        for (int k = 0; k < 4; ++k) RedLane<F, GT, kKeep>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
                     }
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
@@ -1216,7 +1260,7 @@ __device__ __forceinline__ void walk_run_pair(GT* dl, float scale, uint32_t mask
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         if ((((uint32_t)k >> b) & 1u) == leave_bit)
-                            RedLane<F, GT>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
+                            RedLane<F, GT, kKeep>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
                     float old[4][F];
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
@@ -1231,7 +1275,7 @@ __device__ __forceinline__ void walk_run_pair(GT* dl, float scale, uint32_t mask
                 } else {
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        RedLane<F, GT>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
+                        RedLane<F, GT, kKeep>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
 #pragma unroll
                         for (int f = 0; f < F; ++f) acc[k][f] = 0.f;
                     }
@@ -1250,7 +1294,7 @@ __device__ __forceinline__ void walk_run_pair(GT* dl, float scale, uint32_t mask
     }
     if (n > 0) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) RedLane<F, GT>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
+        for (int k = 0; k < 4; ++k) RedLane<F, GT, kKeep>::add(dl + (uint64_t)cidx[k] * F, acc[k]);
     }
 }
 
@@ -1359,13 +1403,6 @@ __device__ __forceinline__ void load_global_entry(const float* p, float* v) {
             v[j] = a.x; v[j + 1] = a.y; v[j + 2] = a.z; v[j + 3] = a.w;
         }
     }
-}
-
-// L2 policy that keeps lines resident (evict-last), for the level's table slice.
-__device__ __forceinline__ uint64_t l2_evict_last_policy() {
-    uint64_t pol;
-    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
 }
 
 // F-wide fp32 / fp16 table entry load with an L2 cache policy.
@@ -1483,7 +1520,7 @@ __global__ void __launch_bounds__(kLevelBlock) backward_kernel_atomic_levels(Lev
             va[f] = cr.w[2 * qq] * g[f];
             vb[f] = cr.w[2 * qq + 1] * g[f];
         }
-        red_pair<F>(dl, cr.idx[2 * qq], cr.idx[2 * qq + 1], va, vb);
+        red_pair<F, true>(dl, cr.idx[2 * qq], cr.idx[2 * qq + 1], va, vb);
     }
 }
 
@@ -1498,7 +1535,7 @@ __global__ void __launch_bounds__(kLevelBlock) backward_kernel_runs_levels(Level
     const int n = (int)min((int64_t)kRun, N - p0);
     const int64_t W = lp.L * F;
     GT* dl = dtable + (uint64_t)l * lp.T * F;
-    walk_run<F>(dl, lp.scale[l], lp.mask, n,
+    walk_run<F, true>(dl, lp.scale[l], lp.mask, n,
                 [&](int j, float* x3) {
                     const float* q = x + (p0 + j) * 3;
                     x3[0] = ld_x(q); x3[1] = ld_x(q + 1); x3[2] = ld_x(q + 2);
@@ -1520,7 +1557,7 @@ __global__ void __launch_bounds__(kLevelBlock) backward_kernel_runs_levels_lanes
     const int64_t W = lp.L * F;
     const uint32_t lane = threadIdx.x & 31;
     GT* dl = dtable + (uint64_t)l * lp.T * F;
-    walk_run_pair<F>(dl, lp.scale[l], lp.mask, n, lane & 1, 3u << (lane & 30),
+    walk_run_pair<F, true>(dl, lp.scale[l], lp.mask, n, lane & 1, 3u << (lane & 30),
                      [&](int j, float* x3) {
                          const float* q = x + (p0 + j) * 3;
                          x3[0] = ld_x(q); x3[1] = ld_x(q + 1); x3[2] = ld_x(q + 2);
