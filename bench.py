@@ -11,7 +11,7 @@ gradient, backward (weighted scatter-add into the fp32 gradient table). The defa
 workload is the 16-level, F=2, T=2^19 grid (N 16->512) on 2^14 rays x 64 stratified
 samples (2^20 points). W warm-up steps, then the K-step loop runs R times back to back so
 that the timed region lasts at least --min-timed-s (all R*K steps timed with CUDA events,
-L2 flushed by a 256 MiB write before every step, outside its events). Rank 0 prints one
+L2 flushed before every step, outside its events: see L2Flush). Rank 0 prints one
 JSON line with the rate, per-kernel rooflines (HBM basis, and the L2 basis against the
 gather / reduction rates the probe kernels measure in the same run), clocks, the other
 workloads as "legs" (forward-only grid on 2^18 uniform points, also under "fwd"; fp16
@@ -326,6 +326,25 @@ class Resident:
         self.hg.hashgrid_destroy(self.handle)
 
 
+class L2Flush:
+    """Evicts the workload's data from L2 before a timed launch, outside its events: writes
+    a 256 MiB buffer (twice the L2), then reads a second 256 MiB buffer. The read evicts
+    the write's dirty lines, so their write-back to HBM happens here rather than inside the
+    next timed launch (measured: it added ~8 us to the 52 us sparse Adam step). L2 is left
+    holding clean lines of the read buffer and none of the workload's data."""
+
+    def __init__(self, device):
+        import torch
+        self.wbuf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.rbuf = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+        self()  # loads the two kernels now, so that no warm-up step pays for it
+        torch.cuda.synchronize(device)
+
+    def __call__(self):
+        self.wbuf.fill_(1)
+        self.rbuf.amax()
+
+
 def loop_repeats(steps: int, step_s: float, min_timed_s: float) -> int:
     """How many times the K-step loop runs back to back in the timed region so that the
     region lasts at least ``min_timed_s`` (at least once)."""
@@ -344,13 +363,13 @@ def time_steps(res: Resident, steps: int, warmup: int, device, sampler=None, min
     import torch
     stream = torch.cuda.current_stream(device)
     sp = stream.cuda_stream
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
 
     def one(evs=None):
         # forward, then zero the gradient, then backward: the zeroed gradient table is
         # still in L2 when the backward's reductions reach it (zeroing before the forward
         # lets the forward's output writes evict it; measured ~2% slower backward)
-        flush.fill_(1)
+        flush()
         if evs:
             evs[0].record(stream)
         res.forward(sp)
@@ -401,12 +420,15 @@ def time_steps(res: Resident, steps: int, warmup: int, device, sampler=None, min
     }
 
 
-def time_e2e(res: Resident, steps: int, warmup: int, device) -> dict:
+def time_e2e(res: Resident, steps: int, warmup: int, device, min_timed_s: float = 0.0) -> dict:
     """End to end through the C ABI from pinned host buffers: per step, copy x (and the
     upstream gradient) host->device, forward, zero the gradient, backward, and copy the
     encoding back to pinned host memory. The gradient table stays on the device for the
     optimizer. Steps are pipelined on three streams with double buffers: the upload of
-    step k+1 and the download of step k-1 overlap step k's kernels (PCIe is full duplex)."""
+    step k+1 and the download of step k-1 overlap step k's kernels (PCIe is full duplex).
+    The timed run is R * K steps, R from the warm-up's wall time (the same on every rank)
+    so that it lasts at least ``min_timed_s``: a stream of steps, whose rate the pipeline's
+    fill and drain (about one upload and one download) distort less the longer it runs."""
     import torch
     hg = res.hg
     s_in, s_comp, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device), torch.cuda.Stream(device)
@@ -447,18 +469,22 @@ def time_e2e(res: Resident, steps: int, warmup: int, device) -> dict:
             oh[b].copy_(od[b], non_blocking=True)
             ev_out[b].record(s_out)
 
+    torch.cuda.synchronize(device)
+    t0 = time.perf_counter()
     for k in range(warmup):
         one(k)
     torch.cuda.synchronize(device)
+    step_s = (time.perf_counter() - t0) / max(warmup, 1)
+    n = steps * int(max_over_ranks(float(loop_repeats(steps, step_s, min_timed_s)), device))
     barrier(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(s_in)
-    for k in range(steps):
+    for k in range(n):
         one(warmup + k)
     e1.record(s_out)
     torch.cuda.synchronize(device)
     ms = max_over_ranks(e0.elapsed_time(e1), device)
-    return {"ms": ms, "h2d": h2d, "d2h": d2h}
+    return {"ms": ms, "h2d": h2d, "d2h": d2h, "steps": n}
 
 
 def time_launches(fn, steps: int, warmup: int, device, before=None) -> float:
@@ -466,14 +492,14 @@ def time_launches(fn, steps: int, warmup: int, device, before=None) -> float:
     calls, each after an L2 flush and the optional untimed ``before``."""
     import torch
     stream = torch.cuda.current_stream(device)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     for _ in range(warmup):
         if before is not None:
             before()
         fn()
     ts = []
     for _ in range(steps):
-        flush.fill_(1)
+        flush()
         if before is not None:
             before()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -836,7 +862,8 @@ def run_b200(args) -> None:
                    "step": "forward + zero dL_dtable + backward" if w.backward else "forward",
                    "modes": {"forward_gather": args.forward_gather, "backward": args.backward_mode,
                              "schedule": args.schedule},
-                   "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                   "l2": "flushed before every timed step, outside the events: a 256 MiB write, then a 256 MiB read "
+                         "that evicts the write's dirty lines",
                    "timed_region": f"the {args.steps}-step loop run {main['loop_repeats']} times back to back "
                                    f"({main['timed_steps']} steps, all timed) so that it lasts >= {args.min_timed_s} s",
                    "phase_ms": main["phase_ms"]},
@@ -871,10 +898,10 @@ def run_b200(args) -> None:
             line["next_rows"]["cpu_oracle"] = cpu_next_rows(w, min(NEXT_ROWS_CPU_SAMPLE, res.N))
 
     if not args.skip_e2e:
-        e = time_e2e(res, args.steps, min(args.warmup, 3), device)
-        launches += args.steps * (2 if w.backward else 1)
-        line["e2e"] = {"value": round(res.N * world * args.steps / (e["ms"] * 1e-3), 1), "unit": UNIT,
-                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+        e = time_e2e(res, args.steps, min(args.warmup, 3), device, args.min_timed_s)
+        launches += e["steps"] * (2 if w.backward else 1)
+        line["e2e"] = {"value": round(res.N * world * e["steps"] / (e["ms"] * 1e-3), 1), "unit": UNIT,
+                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"], "timed_steps": e["steps"],
                        "note": "pinned host x (and upstream grads) -> device, fwd + zero + bwd through "
                                "the C ABI, encoding -> pinned host; the gradient table stays on the device"}
     line["gpu_launches"] = launches
