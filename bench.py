@@ -612,7 +612,7 @@ def stream_bytes_per_point(w: workloads.Workload, kind: str) -> int:
 
 
 def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, kernel: str,
-             l2peaks: dict | None, grad_dtype: str = "f32") -> dict:
+             l2peaks: dict | None, grad_dtype: str = "f32", level_major: bool | None = None) -> dict:
     """Roofline of one kernel launch over ``points`` points (kind "fwd" or "bwd").
 
     HBM (the primary fraction, bound "hbm"): the algorithmic bytes of the launch (x, the
@@ -623,7 +623,8 @@ def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, ke
     hash's access pattern from an L2-resident buffer of the working set's size: x-neighbour
     pairs of F*s-byte entries (fwd) or F-wide fp32 / fp16 contributions (bwd), measured in
     the same run by the probe kernels. The working set is the table (fwd) or gradient
-    (bwd), or one level of it under the level-major schedule (tables above 96 MB).
+    (bwd), or one level of it under the level-major schedule (AUTO for tables above 96 MB;
+    ``level_major`` says which schedule ran when it was chosen explicitly).
     bound_time is the larger of the L2 time and the time of the bytes that must cross HBM
     (all of them for a table larger than L2, else the x / output / upstream-gradient
     rows); frac_bound_time = bound_time / kernel time. Batches more coherent than the
@@ -641,14 +642,16 @@ def roofline(w: workloads.Workload, kind: str, points: int, kernel_ms: float, ke
     hbm_gbs = alg / (kernel_ms * 1e-3) / 1e9
     elem = s if kind == "fwd" else (2 if grad_dtype == "f16" else 4)
     table_bytes = w.L * w.T * w.F * elem
-    level_major = w.L * w.T * w.F * s > L2_RESIDENT_BYTES
+    if level_major is None:
+        level_major = w.L * w.T * w.F * s > L2_RESIDENT_BYTES
     working_set = table_bytes // w.L if level_major else table_bytes
     in_l2 = working_set <= L2_RESIDENT_BYTES
     out = {"bound": "hbm", "kernel": kernel, "kernel_ms": round(kernel_ms, 5), "unit": "GB/s",
            "achieved": round(hbm_gbs, 1), "peak": hbm, "frac": round(hbm_gbs / hbm, 4),
            "traffic": ncu_traffic(kernel, w.name), "algorithmic_bytes_per_launch": alg,
            "peak_source": f"hbm_gbs of {src} peaks"}
-    t_stream = (alg if not (in_l2 and not level_major) else stream_bytes_per_point(w, kind) * points) / (hbm * 1e9)
+    # the table (or gradient) crosses HBM only when it does not fit in L2 as a whole
+    t_stream = (alg if table_bytes > L2_RESIDENT_BYTES else stream_bytes_per_point(w, kind) * points) / (hbm * 1e9)
     t_l2 = 0.0
     if l2peaks is not None and in_l2:
         ops = 8 * w.L * points
@@ -805,6 +808,26 @@ def run_reference(args) -> None:
 LEGS = ("grid_L16F2T19", "half_L16F2T19", "large_L16F4T22")   # timed besides the step's workload
 
 
+def time_level_serial(res: Resident, args, device, l2peaks) -> tuple[dict, int]:
+    """The forward of a table that fits in L2, run level by level (the level-major
+    schedule: one level's table slice is the live working set) instead of point by point
+    (the whole table live): if the point-major forward were losing to L2 capacity, this
+    would be the faster one. Returns the JSON object and the number of timed launches."""
+    import torch
+    hg = res.hg
+    sp = torch.cuda.current_stream(device).cuda_stream
+    steps = min(args.steps, 20)
+    hg.hashgrid_set_option(res.handle, hg.HASHGRID_OPT_SCHEDULE, SCHEDULES["level"])
+    try:
+        ms = time_launches(lambda: res.forward(sp), steps, min(args.warmup, 3), device)
+    finally:
+        hg.hashgrid_set_option(res.handle, hg.HASHGRID_OPT_SCHEDULE, SCHEDULES[args.schedule])
+    return {"schedule": "level", "fwd_ms": round(ms, 5),
+            "rooflines": {"fwd": roofline(res.w, "fwd", res.N, ms, "forward_kernel_levels", l2peaks, level_major=True)},
+            "note": "the same forward with the level-major schedule: one level's table slice live instead of the "
+                    "whole table; if the point-major forward lost to L2 capacity, this one would be faster"}, steps
+
+
 def time_workload(w: workloads.Workload, args, device, rank: int, world: int, l2peaks, min_timed_s: float,
                   sampler=None) -> tuple[dict, Resident, int]:
     """Times one workload's step (forward, or forward + zero + backward) and returns its
@@ -882,6 +905,9 @@ def run_b200(args) -> None:
                 continue
             lw = workloads.WORKLOADS[name]
             obj, lres, n = time_workload(lw, args, device, rank, world, l2peaks, 0.0)
+            if name == FWD_WORKLOAD and args.schedule == "auto":
+                obj["level_serial"], m = time_level_serial(lres, args, device, l2peaks)
+                n += m
             lres.close()
             del lres
             torch.cuda.empty_cache()

@@ -77,6 +77,18 @@ def test_roofline_large_grid_is_hbm_bound_per_level(monkeypatch):
     assert "64MiB" in r["l2"]["peak_source"] and "16-byte" in r["l2"]["access"]
 
 
+def test_roofline_level_serial_schedule(monkeypatch):
+    """A table that fits in L2, run level by level: the L2 term uses one level's slice
+    (4 MB for the default grid, the 32 MiB probe buffer), and the HBM term only the
+    streams, as for the point-major forward."""
+    monkeypatch.setattr(bench, "measured_peaks", lambda: (5000.0, "test"))
+    n, ms = 1 << 18, 0.095
+    r = bench.roofline(W["grid_L16F2T19"], "fwd", n, ms, "forward_kernel_levels", fake_peaks(), level_major=True)
+    assert "32MiB" in r["l2"]["peak_source"] and r["bound_by"] == "l2"
+    p = bench.roofline(W["grid_L16F2T19"], "fwd", n, ms, "forward_kernel", fake_peaks())
+    assert "64MiB" in p["l2"]["peak_source"] and r["frac"] == p["frac"]
+
+
 def test_loop_repeats_reach_the_minimum_timed_region():
     for steps, step_s in [(20, 0.7e-3), (3, 5e-3), (50, 1e-4)]:
         r = bench.loop_repeats(steps, step_s, 1.0)
