@@ -71,8 +71,17 @@ enum hashgrid_status {
     HASHGRID_ERR_ALIGN = 2,        /* a pointer is not 16-byte aligned */
     HASHGRID_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed */
     HASHGRID_ERR_OOM = 4,          /* host allocation of the handle failed */
-    HASHGRID_ERR_DEVICE_CHECK = 5  /* reserved: a device-side range check tripped */
+    HASHGRID_ERR_DEVICE_CHECK = 5  /* checked build only: a device-side range check tripped */
 };
+
+/* The checked build (libhashgrid_checked.so, compiled with -DHASHGRID_CHECKED) tests every
+ * global-memory access of the kernels against the extent of the buffer it belongs to. An
+ * access outside it is skipped (a load reads zero) and the call returns
+ * HASHGRID_ERR_DEVICE_CHECK, naming the buffers in hashgrid_last_error(). Its calls wait for
+ * their kernel, since they read the device status word back. They are meant for one stream
+ * at a time, and they return HASHGRID_ERR_ARG, before any work, on a stream that is being
+ * captured into a CUDA graph. The regular build (libhashgrid.so) has none of this and never
+ * returns HASHGRID_ERR_DEVICE_CHECK. */
 
 /* Parameter limits checked by hashgrid_create. The pages use L = 16 to 32 levels
  * ([Repro-HG] section 5, [Overview-HG] section 2.1) and F = 2 to 4 features. */

@@ -482,6 +482,14 @@ struct CheckBuf {
 template <class Fn>
 int run_checked(cudaStream_t s, std::initializer_list<CheckBuf> bufs, const char* what, Fn&& fn) {
 #ifdef HASHGRID_CHECKED
+    // the status word is read back after the kernel: not possible inside stream capture
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(HASHGRID_ERR_CUDA, "%s: cudaStreamIsCapturing failed", what);
+    }
+    if (cap != cudaStreamCaptureStatusNone)
+        return fail(HASHGRID_ERR_ARG, "%s: the checked build cannot run inside stream capture", what);
     hg::CheckRanges r;
     for (int i = 0; i < hg::kChkRoles; ++i) {
         r.lo[i] = 0;

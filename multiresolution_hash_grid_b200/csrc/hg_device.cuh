@@ -121,6 +121,36 @@ template <int F, typename TT> struct EntryLoad {
 // Point coordinate load (streaming).
 __device__ __forceinline__ float ld_x(const float* p) { return in_bounds<kChkX>(p, 4) ? __ldcs(p) : 0.f; }
 
+// Four consecutive coordinates (streaming); p is 16-byte aligned.
+__device__ __forceinline__ float4 ld_x4(const float* p) {
+    return in_bounds<kChkX>(p, 16) ? __ldcs(reinterpret_cast<const float4*>(p)) : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// Block-wide staging of the n coordinates of a tile, src = x + p0 * D (16-byte aligned: the
+// library takes x 16-byte aligned, and every tile starts at a multiple of 4 points):
+// coalesced float4 loads for the whole groups of four, scalar loads for the tail. put(k, v)
+// stores coordinate k of the tile.
+template <class Put>
+__device__ __forceinline__ void stage_x(const float* __restrict__ src, int n, Put put) {
+    const int n4 = n >> 2;
+    for (int q = threadIdx.x; q < n4; q += blockDim.x) {
+        const float4 v = ld_x4(src + 4 * q);
+        put(4 * q, v.x);
+        put(4 * q + 1, v.y);
+        put(4 * q + 2, v.z);
+        put(4 * q + 3, v.w);
+    }
+    for (int k = 4 * n4 + threadIdx.x; k < n; k += blockDim.x) put(k, ld_x(src + k));
+}
+
+// The same into a contiguous, 16-byte-aligned shared-memory array.
+__device__ __forceinline__ void stage_x(float* xs, const float* __restrict__ src, int n) {
+    const int n4 = n >> 2;
+    for (int q = threadIdx.x; q < n4; q += blockDim.x)
+        *reinterpret_cast<float4*>(xs + 4 * q) = ld_x4(src + 4 * q);
+    for (int k = 4 * n4 + threadIdx.x; k < n; k += blockDim.x) xs[k] = ld_x(src + k);
+}
+
 // ---------------------------------------------------------------------------------------
 // Sector gathers. The x prime is 1, so the two corners that differ only in x, v0 and
 // v0 + 1, hash to (v0 ^ K) and ((v0 + 1) ^ K) for the same K = hash of (y, z): their
@@ -606,7 +636,7 @@ __global__ void __launch_bounds__(512, forward_min_blocks(F, kGather)) forward_k
     const int64_t p0 = (int64_t)blockIdx.x * BP;
     const int nvalid = (int)min((int64_t)BP, N - p0);
 
-    for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = ld_x(x + p0 * 3 + i);
+    stage_x(xs, x + p0 * 3, nvalid * 3);
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -746,6 +776,8 @@ __global__ void __launch_bounds__(512, forward_lanes_min_blocks(F))
     const int64_t p0 = (int64_t)blockIdx.x * BP;
     const int nvalid = (int)min((int64_t)BP, N - p0);
 
+    // scalar loads here: the float4 staging of the other tile kernels measured 1% slower on
+    // uniform points for this kernel (78.7 against 77.9 us per 2^18 points)
     for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = ld_x(x + p0 * 3 + i);
     __syncthreads();
 
@@ -925,7 +957,7 @@ __device__ __forceinline__ void backward_body(const LevelParams& lp, const float
     GroupWarp<FG> grp(reinterpret_cast<char*>(smem + BP * 3 + BP * S), warp);
     if constexpr (kMode != kAtomicOnly) grp.clear(lane);
 
-    for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = ld_x(x + p0 * 3 + i);
+    stage_x(xs, x + p0 * 3, nvalid * 3);
     stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
     __syncthreads();
 
@@ -1104,10 +1136,10 @@ __global__ void __launch_bounds__(256) backward_kernel_runs(LevelParams lp, cons
     const int64_t p0 = (int64_t)blockIdx.x * kRunTile;
     const int nvalid = (int)min((int64_t)kRunTile, N - p0);
 
-    for (int k = threadIdx.x; k < nvalid * 3; k += blockDim.x) {
+    stage_x(x + p0 * 3, nvalid * 3, [&](int k, float v) {
         const int p = k / 3, i = k - 3 * (k / 3);
-        xs[(p / kRun) * XS + (p % kRun) * 3 + i] = ld_x(x + p0 * 3 + k);
-    }
+        xs[(p / kRun) * XS + (p % kRun) * 3 + i] = v;
+    });
     {
         constexpr int V = F < 4 ? F : 4;
         const int per_row = W / V;
@@ -1316,10 +1348,10 @@ __global__ void __launch_bounds__(256) backward_kernel_runs_lanes(LevelParams lp
     const int64_t p0 = (int64_t)blockIdx.x * kRunTile;
     const int nvalid = (int)min((int64_t)kRunTile, N - p0);
 
-    for (int k = threadIdx.x; k < nvalid * 3; k += blockDim.x) {
+    stage_x(x + p0 * 3, nvalid * 3, [&](int k, float v) {
         const int p = k / 3, i = k - 3 * (k / 3);
-        xs[(p / kRun) * XS + (p % kRun) * 3 + i] = ld_x(x + p0 * 3 + k);
-    }
+        xs[(p / kRun) * XS + (p % kRun) * 3 + i] = v;
+    });
     {
         constexpr int V = F < 4 ? F : 4;
         const int per_row = W / V;
@@ -1594,7 +1626,7 @@ __global__ void __launch_bounds__(512, F <= 2 ? 3 : 2) backward_input_kernel(Lev
     const int64_t p0 = (int64_t)blockIdx.x * BP;
     const int nvalid = (int)min((int64_t)BP, N - p0);
 
-    for (int i = threadIdx.x; i < nvalid * 3; i += blockDim.x) xs[i] = ld_x(x + p0 * 3 + i);
+    stage_x(xs, x + p0 * 3, nvalid * 3);
     stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
     __syncthreads();
 

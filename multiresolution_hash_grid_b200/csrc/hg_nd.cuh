@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(512) forward_kernel(LevelParams lp, const floa
     float* os = smem + kTile * D;
     const int64_t p0 = (int64_t)blockIdx.x * kTile;
     const int nvalid = (int)min((int64_t)kTile, N - p0);
-    for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) xs[i] = ld_x(x + p0 * D + i);
+    stage_x(xs, x + p0 * D, nvalid * D);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     if constexpr (kLanes) {
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(512) backward_kernel(LevelParams lp, const flo
     float* gs = smem + kTile * D;
     const int64_t p0 = (int64_t)blockIdx.x * kTile;
     const int nvalid = (int)min((int64_t)kTile, N - p0);
-    for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) xs[i] = ld_x(x + p0 * D + i);
+    stage_x(xs, x + p0 * D, nvalid * D);
     stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(512) backward_input_kernel(LevelParams lp, con
     float* part = gs + kTile * S;  // [L][D][kTile]
     const int64_t p0 = (int64_t)blockIdx.x * kTile;
     const int nvalid = (int)min((int64_t)kTile, N - p0);
-    for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) xs[i] = ld_x(x + p0 * D + i);
+    stage_x(xs, x + p0 * D, nvalid * D);
     stage_rows_in<(F < 4 ? F : 4)>(gs, dout, p0, nvalid, W, S);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;

@@ -78,3 +78,39 @@ def test_a_tripped_check_is_reported_and_the_access_skipped():
     r = subprocess.run([sys.executable, "-c", TRIP], cwd=ROOT, env=checked_env(), capture_output=True, text=True,
                        timeout=300)
     assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
+
+
+CAPTURE = r"""
+import numpy as np, torch, multiresolution_hash_grid_b200 as hg, workloads
+assert "checked" in hg.hashgrid_version()
+g = hg.HashGrid(4, 2, 10, 2, 16)
+rng = np.random.default_rng(4)
+x = torch.from_numpy(workloads.uniform_points(rng, 500)).cuda()
+t = torch.from_numpy(workloads.table_values(rng, 4, 1024, 2)).cuda()
+want = g.forward(x, t)
+torch.cuda.synchronize()
+out = torch.zeros((500, 8), device="cuda")
+s = torch.cuda.Stream()
+graph = torch.cuda.CUDAGraph()
+codes = []
+with torch.cuda.graph(graph, stream=s):
+    codes.append(hg.lib.hashgrid_forward(g.handle, x.data_ptr(), 500, t.data_ptr(), out.data_ptr(),
+                                         torch.cuda.current_stream().cuda_stream))
+assert codes == [hg.HASHGRID_ERR_ARG], codes
+assert "stream capture" in hg.hashgrid_last_error(), hg.hashgrid_last_error()
+graph.replay()                      # the call issued nothing into the graph
+torch.cuda.synchronize()
+assert bool(torch.all(out == 0))
+assert torch.equal(g.forward(x, t), want)   # eager calls still work
+print("ok")
+"""
+
+
+@pytest.mark.gpu
+def test_stream_capture_is_refused_before_any_work():
+    """The checked build reads its status word back after every kernel, which stream
+    capture does not allow: a call on a capturing stream returns HASHGRID_ERR_ARG and
+    issues nothing, and the capture and later eager calls are unaffected."""
+    r = subprocess.run([sys.executable, "-c", CAPTURE], cwd=ROOT, env=checked_env(), capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
