@@ -809,10 +809,11 @@ LEGS = ("grid_L16F2T19", "half_L16F2T19", "large_L16F4T22")   # timed besides th
 
 
 def time_level_serial(res: Resident, args, device, l2peaks) -> tuple[dict, int]:
-    """The forward of a table that fits in L2, run level by level (the level-major
-    schedule: one level's table slice is the live working set) instead of point by point
-    (the whole table live): if the point-major forward were losing to L2 capacity, this
-    would be the faster one. Returns the JSON object and the number of timed launches."""
+    """The forward of a table that fits in L2, run level-major (one pass per group of
+    levels whose reachable entries fit in 32 MB: the group's slices are the live working
+    set) instead of point by point (the whole table live): if the point-major forward were
+    losing to L2 capacity, this would be the faster one. Returns the JSON object and the
+    number of timed launches."""
     import torch
     hg = res.hg
     sp = torch.cuda.current_stream(device).cuda_stream
@@ -824,8 +825,9 @@ def time_level_serial(res: Resident, args, device, l2peaks) -> tuple[dict, int]:
         hg.hashgrid_set_option(res.handle, hg.HASHGRID_OPT_SCHEDULE, SCHEDULES[args.schedule])
     return {"schedule": "level", "fwd_ms": round(ms, 5),
             "rooflines": {"fwd": roofline(res.w, "fwd", res.N, ms, "forward_kernel_levels", l2peaks, level_major=True)},
-            "note": "the same forward with the level-major schedule: one level's table slice live instead of the "
-                    "whole table; if the point-major forward lost to L2 capacity, this one would be faster"}, steps
+            "note": "the same forward with the level-major schedule: a group of levels (at most 32 MB of entries "
+                    "reachable) live instead of the whole table; if the point-major forward lost to L2 capacity, "
+                    "this one would be faster"}, steps
 
 
 def time_workload(w: workloads.Workload, args, device, rank: int, world: int, l2peaks, min_timed_s: float,

@@ -249,6 +249,33 @@ bool run_lanes(const hashgrid_s* h) {
 // Level-major when asked, or (AUTO) when the whole table is larger than most of L2.
 constexpr size_t kLevelMajorTableBytes = 96u << 20;
 
+// Level groups of the level-major lane-pair kernels. A level's points in the unit cube reach
+// at most min(T, (N_l + 2)^3) entries, so the coarse levels of a large table touch only a
+// few MB of their slices. Consecutive levels are grouped while the entries they can reach
+// (counted at 4F bytes, the fp32 gradient's width) stay within 32 MB, a quarter of the L2;
+// a level above that is a group of its own. One pass per group then reads x and writes the
+// output rows once for all its levels. (1 GiB grid, L = 16, F = 4: levels 0-5 reach 26.5 MB
+// together and form one group, levels 6-15 one group each.)
+constexpr double kLevelGroupBytes = 32.0 * (1 << 20);
+
+void compute_level_groups(hashgrid_s* h) {
+    const double T = (double)((uint64_t)1 << h->log2T);
+    int g = 0;
+    double acc = 0.0;
+    h->lp.group_lo[0] = 0;
+    for (int l = 0; l < h->L; ++l) {
+        const double v = (double)h->res[l] + 2.0;
+        const double bytes = std::min(T, v * v * v) * h->F * 4.0;
+        if (l > 0 && acc + bytes > kLevelGroupBytes) {
+            h->lp.group_lo[++g] = l;
+            acc = 0.0;
+        }
+        acc += bytes;
+    }
+    h->lp.group_lo[++g] = h->L;
+    h->lp.ngroups = g;
+}
+
 bool level_major(const hashgrid_s* h) {
     if (h->schedule == HASHGRID_SCHEDULE_LEVEL_MAJOR) return true;
     if (h->schedule == HASHGRID_SCHEDULE_POINT_MAJOR) return false;
@@ -260,7 +287,7 @@ template <int F, typename TT>
 int launch_forward_levels(const hashgrid_s* h, const float* x, int64_t N, const void* table, float* out,
                           int gather, cudaStream_t s) {
     if (gather == hg::kGatherLanes) {  // two threads per point
-        const dim3 grid((unsigned)((2 * N + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
+        const dim3 grid((unsigned)((2 * N + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->lp.ngroups);
         hg::forward_kernel_levels_lanes<F, TT><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, N, static_cast<const TT*>(table), out);
         return launch_status("forward");
     }
@@ -277,7 +304,7 @@ int launch_backward_levels(const hashgrid_s* h, const float* x, const float* dou
     if constexpr (F <= 4) {
         if (run_lanes(h)) {
             const int64_t runs = (N + hg::kRun - 1) / hg::kRun;
-            const dim3 grid((unsigned)((2 * runs + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->L);
+            const dim3 grid((unsigned)((2 * runs + hg::kLevelBlock - 1) / hg::kLevelBlock), (unsigned)h->lp.ngroups);
             hg::backward_kernel_runs_levels_lanes<F, GT><<<grid, hg::kLevelBlock, 0, s>>>(h->lp, x, dout, N, dtable);
             return launch_status("backward");
         }
@@ -573,6 +600,7 @@ int hashgrid_create(int L, int F, int log2T, int N_min, int N_max, int dtype, ha
     h->lp.T = (uint64_t)1 << log2T;
     h->lp.mask = (uint32_t)(h->lp.T - 1);
     for (int l = 0; l < L; ++l) h->lp.scale[l] = (float)h->res[l];
+    compute_level_groups(h);
     *out = h;
     return ok();
 }

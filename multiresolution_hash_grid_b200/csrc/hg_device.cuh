@@ -37,6 +37,11 @@ struct LevelParams {
     uint32_t mask;            // T - 1
     int L;
     uint64_t T;               // entries per level table
+    // Level groups of the level-major lane-pair kernels: group g is levels
+    // [group_lo[g], group_lo[g + 1]), consecutive levels whose table entries that points in
+    // the unit cube can reach fit in a shared L2 budget together (one pass per group).
+    int ngroups;
+    int group_lo[kMaxLevels + 1];
 };
 
 // Shared-memory row stride (in floats) of a staged [BP, L*F] tile. The padding keeps the
@@ -1503,33 +1508,38 @@ __global__ void __launch_bounds__(kLevelBlock) forward_kernel_levels(LevelParams
     store_global_entry<F>(out + p * (int64_t)(lp.L * F) + l * F, o);
 }
 
-// Level-major forward with lane pairs: two threads per point at level blockIdx.y.
+// Level-major forward with lane pairs: two threads per point for the levels of group
+// blockIdx.y, in order (x is read once per group, and a group's output pieces of a row
+// are written back to back, so its sectors leave L2 whole).
 template <int F, typename TT>
 __global__ void __launch_bounds__(kLevelBlock) forward_kernel_levels_lanes(LevelParams lp, const float* __restrict__ x,
                                                                           int64_t N, const TT* __restrict__ table,
                                                                           float* __restrict__ out) {
-    const int l = blockIdx.y;
+    const int g = blockIdx.y;
     const int64_t p = ((int64_t)blockIdx.x * kLevelBlock + threadIdx.x) >> 1;
     if (p >= N) return;  // both lanes of a pair return together
     const uint32_t lane = threadIdx.x & 31;
     const uint32_t d0 = lane & 1;
     const unsigned pair = 3u << (lane & 30);
-    HalfCorners hc;
-    locate_half(ld_x(x + p * 3), ld_x(x + p * 3 + 1), ld_x(x + p * 3 + 2), lp.scale[l], lp.mask, d0, hc);
-    const TT* tl = table + (uint64_t)l * lp.T * F;
+    const float x0 = ld_x(x + p * 3), x1 = ld_x(x + p * 3 + 1), x2 = ld_x(x + p * 3 + 2);
     const uint64_t pol = l2_evict_last_policy();
-    float e[4][F];
+    for (int l = lp.group_lo[g]; l < lp.group_lo[g + 1]; ++l) {
+        HalfCorners hc;
+        locate_half(x0, x1, x2, lp.scale[l], lp.mask, d0, hc);
+        const TT* tl = table + (uint64_t)l * lp.T * F;
+        float e[4][F];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) load_entry_policy<F, TT>(tl + (uint64_t)hc.idx[k] * F, e[k], pol);
-    float o[F];
+        for (int k = 0; k < 4; ++k) load_entry_policy<F, TT>(tl + (uint64_t)hc.idx[k] * F, e[k], pol);
+        float o[F];
 #pragma unroll
-    for (int f = 0; f < F; ++f) {
-        float acc = hc.w[0] * e[0][f];
+        for (int f = 0; f < F; ++f) {
+            float acc = hc.w[0] * e[0][f];
 #pragma unroll
-        for (int k = 1; k < 4; ++k) acc = fmaf(hc.w[k], e[k][f], acc);
-        o[f] = acc + __shfl_xor_sync(pair, acc, 1);
+            for (int k = 1; k < 4; ++k) acc = fmaf(hc.w[k], e[k][f], acc);
+            o[f] = acc + __shfl_xor_sync(pair, acc, 1);
+        }
+        store_half<F, true>(out + p * (int64_t)(lp.L * F) + l * F, o, d0);
     }
-    store_half<F, true>(out + p * (int64_t)(lp.L * F) + l * F, o, d0);
 }
 
 template <int F, typename GT>
@@ -1575,26 +1585,29 @@ __global__ void __launch_bounds__(kLevelBlock) backward_kernel_runs_levels(Level
                 [&](int j, float* g) { load_global_entry<F>(dout + (p0 + j) * W + l * F, g); });
 }
 
-// Level-major lane-pair run walk: two threads per run of kRun consecutive points at level
-// blockIdx.y.
+// Level-major lane-pair run walk: two threads per run of kRun consecutive points, walked at
+// each level of group blockIdx.y in turn (the run's x and upstream-gradient rows are read
+// from HBM for the group's first level and from the caches for the others).
 template <int F, typename GT>
 __global__ void __launch_bounds__(kLevelBlock) backward_kernel_runs_levels_lanes(LevelParams lp,
                                                                                 const float* __restrict__ x,
                                                                                 const float* __restrict__ dout,
                                                                                 int64_t N, GT* __restrict__ dtable) {
-    const int l = blockIdx.y;
+    const int grp = blockIdx.y;
     const int64_t p0 = (((int64_t)blockIdx.x * kLevelBlock + threadIdx.x) >> 1) * kRun;
     if (p0 >= N) return;  // both lanes of a pair return together
     const int n = (int)min((int64_t)kRun, N - p0);
     const int64_t W = lp.L * F;
     const uint32_t lane = threadIdx.x & 31;
-    GT* dl = dtable + (uint64_t)l * lp.T * F;
-    walk_run_pair<F, true>(dl, lp.scale[l], lp.mask, n, lane & 1, 3u << (lane & 30),
-                     [&](int j, float* x3) {
-                         const float* q = x + (p0 + j) * 3;
-                         x3[0] = ld_x(q); x3[1] = ld_x(q + 1); x3[2] = ld_x(q + 2);
-                     },
-                     [&](int j, float* g) { load_global_entry<F>(dout + (p0 + j) * W + l * F, g); });
+    for (int l = lp.group_lo[grp]; l < lp.group_lo[grp + 1]; ++l) {
+        GT* dl = dtable + (uint64_t)l * lp.T * F;
+        walk_run_pair<F, true>(dl, lp.scale[l], lp.mask, n, lane & 1, 3u << (lane & 30),
+                               [&](int j, float* x3) {
+                                   const float* q = x + (p0 + j) * 3;
+                                   x3[0] = ld_x(q); x3[1] = ld_x(q + 1); x3[2] = ld_x(q + 2);
+                               },
+                               [&](int j, float* g) { load_global_entry<F>(dout + (p0 + j) * W + l * F, g); });
+    }
 }
 
 // ---------------------------------------------------------------------------------------
