@@ -323,10 +323,13 @@ int launch_backward_levels(const hashgrid_s* h, const float* x, const float* dou
 template <int F, typename GT = float>
 int launch_backward_runs(const hashgrid_s* h, const float* x, const float* dout, int64_t N,
                          GT* dtable, cudaStream_t s) {
-    auto k = run_lanes(h) ? hg::backward_kernel_runs_lanes<F, GT> : hg::backward_kernel_runs<F, GT>;
-    const size_t smem = hg::run_smem_bytes(h->L, F);
+    const bool lanes = run_lanes(h);
+    auto k = lanes ? hg::backward_kernel_runs_lanes<F, GT> : hg::backward_kernel_runs<F, GT>;
+    const size_t smem = lanes ? hg::run_smem_bytes(h->L, F, hg::kRunPairTile / hg::kRunPair, hg::kRunPair)
+                              : hg::run_smem_bytes(h->L, F);
     if (int rc = prepare_smem(k, smem)) return rc;
-    const unsigned blocks = (unsigned)((N + hg::kRunTile - 1) / hg::kRunTile);
+    const int64_t tile = lanes ? hg::kRunPairTile : hg::kRunTile;
+    const unsigned blocks = (unsigned)((N + tile - 1) / tile);
     k<<<blocks, 256, smem, s>>>(h->lp, x, dout, N, dtable);
     return launch_status("backward");
 }

@@ -1046,14 +1046,21 @@ __global__ void __launch_bounds__(256, F == 4 ? 2 : 3) backward_kernel_grouped(L
 // Shared memory: x and the upstream-gradient rows, grouped by run with strides chosen so
 // that the lanes' row reads (lane = run) fall in distinct banks.
 // ---------------------------------------------------------------------------------------
-constexpr int kRun = 8;
-constexpr int kRunTile = 32 * kRun;
+constexpr int kRun = 8;                 // one-lane and level-major walks
+constexpr int kRunTile = 32 * kRun;     // one-lane tile: a run per lane of a warp
+// Lane-pair walks (backward_kernel_runs_lanes) take runs of 16 points, 16 runs per 256-point
+// tile: at coarse levels a run's end flushes its corners even when the next sample shares
+// the voxel, and runs of 16 halve those flushes (rays: 345 against 352 us). The level-major
+// walk keeps runs of 8 (runs of 16 left too few lane pairs in flight there: 3.01 against
+// 2.66 ms on the 1 GiB grid).
+constexpr int kRunPair = 16;
+constexpr int kRunPairTile = 256;
 
-__host__ __device__ constexpr int run_x_stride() { return kRun * 3 + 1; }
+__host__ __device__ constexpr int run_x_stride(int run = kRun) { return run * 3 + 1; }
 __host__ __device__ constexpr int run_row_stride(int L, int F) { return L * F + row_pad(F); }
-__host__ __device__ constexpr int run_g_stride(int L, int F) { return kRun * run_row_stride(L, F) + F; }
-__host__ __device__ constexpr size_t run_smem_bytes(int L, int F) {
-    return sizeof(float) * ((size_t)32 * run_x_stride() + (size_t)32 * run_g_stride(L, F));
+__host__ __device__ constexpr int run_g_stride(int L, int F, int run = kRun) { return run * run_row_stride(L, F) + F; }
+__host__ __device__ constexpr size_t run_smem_bytes(int L, int F, int runs = kRunTile / kRun, int run = kRun) {
+    return sizeof(float) * ((size_t)runs * run_x_stride(run) + (size_t)runs * run_g_stride(L, F, run));
 }
 
 template <int F, bool kKeep = false, typename GT>
@@ -1335,8 +1342,8 @@ __device__ __forceinline__ void walk_run_pair(GT* dl, float scale, uint32_t mask
     }
 }
 
-// Block: kRunTile points (32 runs of kRun) and 8 warps, shared memory as backward_kernel_runs;
-// a warp item is 16 runs at one level (a lane pair per run).
+// Block: kRunPairTile points (16 runs of kRunPair) and 8 warps, shared memory laid out as in
+// backward_kernel_runs; a warp item is 16 runs at one level (a lane pair per run).
 template <int F, typename GT>
 __global__ void __launch_bounds__(256) backward_kernel_runs_lanes(LevelParams lp, const float* __restrict__ x,
                                                                  const float* __restrict__ dout, int64_t N,
@@ -1346,16 +1353,18 @@ __global__ void __launch_bounds__(256) backward_kernel_runs_lanes(LevelParams lp
     const int L = lp.L;
     const int W = L * F;
     const int S = run_row_stride(L, F);
-    const int G = run_g_stride(L, F);
-    constexpr int XS = run_x_stride();
+    constexpr int R = kRunPair;                   // points per run
+    constexpr int NR = kRunPairTile / kRunPair;   // runs per tile
+    const int G = run_g_stride(L, F, R);
+    constexpr int XS = run_x_stride(R);
     float* xs = smem;
-    float* gs = smem + 32 * XS;
-    const int64_t p0 = (int64_t)blockIdx.x * kRunTile;
-    const int nvalid = (int)min((int64_t)kRunTile, N - p0);
+    float* gs = smem + NR * XS;
+    const int64_t p0 = (int64_t)blockIdx.x * kRunPairTile;
+    const int nvalid = (int)min((int64_t)kRunPairTile, N - p0);
 
     stage_x(x + p0 * 3, nvalid * 3, [&](int k, float v) {
         const int p = k / 3, i = k - 3 * (k / 3);
-        xs[(p / kRun) * XS + (p % kRun) * 3 + i] = v;
+        xs[(p / R) * XS + (p % R) * 3 + i] = v;
     });
     {
         constexpr int V = F < 4 ? F : 4;
@@ -1364,7 +1373,7 @@ __global__ void __launch_bounds__(256) backward_kernel_runs_lanes(LevelParams lp
         for (int k = threadIdx.x; k < nvalid * per_row; k += blockDim.x) {
             const int row = k / per_row;
             const int col = (k - row * per_row) * V;
-            float* dst = gs + (row / kRun) * G + (row % kRun) * S + col;
+            float* dst = gs + (row / R) * G + (row % R) * S + col;
             const float* src = base + (int64_t)row * W + col;
             if (!in_bounds<kChkDout>(src, 4 * V)) continue;
             if constexpr (V == 4) {
@@ -1382,11 +1391,11 @@ __global__ void __launch_bounds__(256) backward_kernel_runs_lanes(LevelParams lp
     const int nwarps = blockDim.x >> 5;
     const uint32_t d0 = lane & 1;
     const unsigned pair = 3u << (lane & 30);
-    for (int it = warp; it < 2 * L; it += nwarps) {
+    for (int it = warp; it < (NR / 16) * L; it += nwarps) {
         const int h = it / L;
         const int l = it - h * L;
         const int run = h * 16 + (lane >> 1);
-        const int jmax = min(kRun, nvalid - run * kRun);  // the same for both lanes of a pair
+        const int jmax = min(R, nvalid - run * R);  // the same for both lanes of a pair
         GT* dl = dtable + (uint64_t)l * lp.T * F;
         walk_run_pair<F>(dl, lp.scale[l], lp.mask, jmax, d0, pair,
                          [&](int j, float* x3) {
