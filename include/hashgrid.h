@@ -294,7 +294,7 @@ const char *hashgrid_last_error(void);
  *     the L1 fetches a shared sector once for both threads. The pair adds its partial sums;
  *     applies to both schedules;
  *   HASHGRID_GATHER_AUTO: LANES (measured fastest on every workload: per 2^20 ray samples
- *     225 us against 250 us for CORNER, per 2^18 uniform points 81 against 95 us).
+ *     221 us against 250 us for CORNER, per 2^18 uniform points 78 against 95 us).
  * HASHGRID_OPT_BACKWARD_MODE -- how the backward pass reduces into dL_dtable:
  *   HASHGRID_BACKWARD_ATOMIC: each (point, level) reduces its 8 corner contributions, the
  *     two x-corners merged into one 16-byte reduction when they share an aligned unit;
@@ -313,19 +313,24 @@ const char *hashgrid_last_error(void);
  *   HASHGRID_BACKWARD_RUN_LANES: RUN_MERGE with two threads per run, thread d keeping the
  *     sums of the 4 corners with x offset d, each corner reduced on its own (F-wide);
  *     x-neighbouring corners, which usually share a sector (the x prime is 1), are reduced
- *     by the same instruction. Needs F <= 4. The schedule option applies;
+ *     by the same instruction. Runs are 16 points long under the point-major schedule and
+ *     8 under the level-major one. Needs F <= 4. The schedule option applies;
  *   HASHGRID_BACKWARD_AUTO: RUN_LANES for F <= 4 (measured fastest on every workload: per
- *     2^20 ray samples 356 us against 424 us for RUN_MERGE, per 2^22 uniform points 1.74
+ *     2^20 ray samples 345 us against 424 us for RUN_MERGE, per 2^22 uniform points 1.74
  *     against 2.10 ms), ATOMIC for F = 8.
  * HASHGRID_OPT_SCHEDULE -- the order in which (point, level) pairs are visited:
  *   HASHGRID_SCHEDULE_POINT_MAJOR: a block handles all levels of a tile of points (best
  *     when the table fits in L2: the x and upstream-gradient rows are read once and the
  *     output rows are written whole);
- *   HASHGRID_SCHEDULE_LEVEL_MAJOR: blocks sweep all points for level 0, then level 1, ...,
- *     so one level's table slice (and gradient slice) stays in L2 while every point
- *     visits it (best for tables much larger than L2; x is read once per level). The
- *     forward pass then gathers with lane pairs (AUTO, LANES) or per corner (any other
- *     gather option), and the warp-dedup backward modes keep their point-major schedule;
+ *   HASHGRID_SCHEDULE_LEVEL_MAJOR: blocks sweep all points for the first group of levels,
+ *     then the next group, ..., so the group's table slices (and gradient slices) stay in
+ *     L2 while every point visits them (best for tables much larger than L2). A group is a
+ *     run of consecutive levels whose entries reachable from the unit cube,
+ *     min(T, (N_l + 2)^3) per level at 4F bytes, fit in 32 MB together: the coarse levels
+ *     of a large table share one pass, the fine levels have one pass each; x is read once
+ *     per group. The forward pass then gathers with lane pairs (AUTO, LANES) or per corner
+ *     (any other gather option), whose kernels take one level per pass; the warp-dedup
+ *     backward modes keep their point-major schedule;
  *   HASHGRID_SCHEDULE_AUTO: LEVEL_MAJOR when the table is larger than 96 MB, else
  *     POINT_MAJOR.
  * Returns HASHGRID_ERR_ARG for an unknown option or value.
