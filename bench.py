@@ -808,7 +808,7 @@ def run_reference(args) -> None:
 LEGS = ("grid_L16F2T19", "half_L16F2T19", "large_L16F4T22")   # timed besides the step's workload
 
 
-def time_level_serial(res: Resident, args, device, l2peaks) -> tuple[dict, int]:
+def time_level_major(res: Resident, args, device, l2peaks) -> tuple[dict, int]:
     """The forward of a table that fits in L2, run level-major (one pass per group of
     levels whose reachable entries fit in 32 MB: the group's slices are the live working
     set) instead of point by point (the whole table live): if the point-major forward were
@@ -908,7 +908,7 @@ def run_b200(args) -> None:
             lw = workloads.WORKLOADS[name]
             obj, lres, n = time_workload(lw, args, device, rank, world, l2peaks, 0.0)
             if name == FWD_WORKLOAD and args.schedule == "auto":
-                obj["level_serial"], m = time_level_serial(lres, args, device, l2peaks)
+                obj["level_major"], m = time_level_major(lres, args, device, l2peaks)
                 n += m
             lres.close()
             del lres

@@ -77,7 +77,7 @@ def test_roofline_large_grid_is_hbm_bound_per_level(monkeypatch):
     assert "64MiB" in r["l2"]["peak_source"] and "16-byte" in r["l2"]["access"]
 
 
-def test_roofline_level_serial_schedule(monkeypatch):
+def test_roofline_level_major_schedule(monkeypatch):
     """A table that fits in L2, run level by level: the L2 term uses one level's slice
     (4 MB for the default grid, the 32 MiB probe buffer), and the HBM term only the
     streams, as for the point-major forward."""
