@@ -1,17 +1,26 @@
-"""Seeded random configurations against the oracle: per seed a random dimension D (2, 3 or
+"""Seeded random configurations against the oracle, for every entry point.
+
+Encoding (indices, forward, fp32 and fp16 backward, dL/dx): per seed a random dimension D (2, 3 or
 4), level count, feature width, table size, resolution range, table dtype, forward gather,
 backward reduction mode and schedule, and a random point count (1 to 700, so most batches
 end in a ragged tile) whose first rows sit on the cube's faces, just inside its upper face
 or outside it. Every entry point is held to the bars of the fixed-shape parity tests:
 indices bit-exact; forward within rtol * sum_c w_c |e_c|; fp32 gradients within 1e-5
 relative L2 per level; fp16 gradients within the fp16 accumulation model; dL/dx within
-1e-5 of its absolute-term bound (scaled by 2^(D-3) for D > 3: twice the corners per level)."""
+1e-5 of its absolute-term bound (scaled by 2^(D-3) for D > 3: twice the corners per level).
+
+Sparse Adam: random levels, widths, table sizes, dtypes, gradient sparsity, step counts and
+the fused clear, each step against the oracle's step from the GPU's state (the bars of
+run_adam_steps). Encoding + MLP: every input width the MLP takes (L * F = 16, 32, 48, 64)
+with F from 1 to 8, random grids, dtypes and gathers, and point counts that leave ragged
+128-point tiles, against the oracle within the propagated bf16 bound of check_mlp."""
 import numpy as np
 import pytest
 
 import oracle
 import workloads
-from tests.test_parity import FWD_RTOL, THREADS, check_gradient, check_half_gradient, dev
+from tests.test_parity import (FWD_RTOL, THREADS, check_gradient, check_half_gradient, check_mlp, dev, mlp_weights,
+                               run_adam_steps)
 
 torch = pytest.importorskip("torch")
 
@@ -112,3 +121,65 @@ def test_configurations_cover_every_option():
     assert {c["gather"] for c in nd} == {"auto", "corner", "lanes"}
     assert {c["backward"] for c in nd} == {"auto", "atomic", "run_lanes"}
     assert {c["dtype"] for c in cs} == {"f32", "f16"} and {c["F"] for c in cs} == {1, 2, 4, 8}
+
+
+def adam_config(seed):
+    rng = np.random.default_rng(3000 + seed)
+    return dict(dtype=str(rng.choice(["f32", "f16"])), zero_grad=bool(rng.integers(0, 2)),
+                L=int(rng.integers(2, 9)), F=int(rng.choice([1, 2, 4, 8])), log2T=int(rng.integers(4, 15)),
+                steps=int(rng.integers(1, 5)), zero_frac=float(rng.choice([0.0, 0.5, 0.9, 0.99])))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed", range(16))
+def test_random_adam(seed):
+    c = adam_config(seed)
+    run_adam_steps(c["dtype"], c["zero_grad"], c["L"], c["F"], c["log2T"], c["steps"], c["zero_frac"], 4000 + seed)
+
+
+def mlp_config(seed):
+    rng = np.random.default_rng(5000 + seed)
+    K = int(rng.choice([16, 32, 48, 64]))
+    F = int(rng.choice([f for f in (1, 2, 4, 8) if K % f == 0 and K // f <= 32]))
+    L = K // F
+    n_min = int(rng.integers(2, 40))
+    n_max = n_min if L == 1 else int(rng.integers(n_min, 3000))
+    return dict(L=L, F=F, log2T=int(rng.integers(4, 17)), N_min=n_min, N_max=n_max,
+                dtype=str(rng.choice(["f32", "f16"])), gather=str(rng.choice(["auto", "corner"])),
+                n=int(rng.integers(1, 700)))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed", range(16))
+def test_random_mlp(seed):
+    import multiresolution_hash_grid_b200 as hg
+    c = mlp_config(seed)
+    L, F, log2T, n = c["L"], c["F"], c["log2T"], c["n"]
+    f16 = c["dtype"] == "f16"
+    grid = hg.HashGrid(L, F, log2T, c["N_min"], c["N_max"], hg.HASHGRID_F16 if f16 else hg.HASHGRID_F32,
+                       forward_gather=GATHER[c["gather"]])
+    og = oracle.Grid(L, F, log2T, c["N_min"], c["N_max"], oracle.F16 if f16 else oracle.F32)
+    rng = np.random.default_rng(6000 + seed)
+    table = (rng.standard_normal((L, 2**log2T, F)) * 0.3).astype(np.float16 if f16 else np.float32)
+    x = rng.random((n, 3), dtype=np.float32)
+    k = min(n, 8)
+    x[:k] = EDGE[rng.integers(0, len(EDGE), size=(k, 3))]
+    wts = mlp_weights(rng, L * F)
+    y = torch.full((n, 4), float("nan"), device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    hg.hashgrid_mlp_forward(grid.handle, dev(x), n, dev(table), *[dev(w) for w in wts], y, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, c
+    check_mlp(og, x, table, wts, y.cpu().numpy())
+
+
+def test_adam_and_mlp_configurations_cover_the_options():
+    """Host check: the Adam seeds reach both dtypes, both clear settings, every width and
+    a dense and a nearly empty gradient; the MLP seeds every input width, F = 1..8, both
+    dtypes and both producer forms."""
+    a = [adam_config(s) for s in range(16)]
+    assert {c["dtype"] for c in a} == {"f32", "f16"} and {c["zero_grad"] for c in a} == {True, False}
+    assert {c["F"] for c in a} == {1, 2, 4, 8} and {0.0, 0.99} <= {c["zero_frac"] for c in a}
+    m = [mlp_config(s) for s in range(16)]
+    assert {c["L"] * c["F"] for c in m} == {16, 32, 48, 64} and {c["F"] for c in m} == {1, 2, 4, 8}
+    assert {c["dtype"] for c in m} == {"f32", "f16"} and {c["gather"] for c in m} == {"auto", "corner"}
