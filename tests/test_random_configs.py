@@ -183,3 +183,69 @@ def test_adam_and_mlp_configurations_cover_the_options():
     m = [mlp_config(s) for s in range(16)]
     assert {c["L"] * c["F"] for c in m} == {16, 32, 48, 64} and {c["F"] for c in m} == {1, 2, 4, 8}
     assert {c["dtype"] for c in m} == {"f32", "f16"} and {c["gather"] for c in m} == {"auto", "corner"}
+
+
+def level_config(seed):
+    rng = np.random.default_rng(7000 + seed)
+    L = int(rng.integers(8, 15))
+    n_min = int(rng.integers(2, 40))
+    return dict(L=L, F=int(rng.choice([2, 4])), log2T=int(rng.integers(19, 21)), N_min=n_min,
+                N_max=int(rng.integers(400, 3000)), dtype=str(rng.choice(["f32", "f16"])),
+                gather=str(rng.choice(["auto", "corner"])), backward=str(rng.choice(["auto", "atomic", "runs"])),
+                n=int(rng.integers(1, 700)))
+
+
+def level_groups(c):
+    """The level-major schedule's grouping rule (consecutive levels while their reachable
+    entries, min(T, (N_l + 2)^3) at 4F bytes, stay within 32 MB), restated to check that
+    the seeds below reach several groups."""
+    lo, acc = [0], 0.0
+    for l, r in enumerate(oracle.resolutions(c["L"], c["N_min"], c["N_max"])):
+        b = min(2.0 ** c["log2T"], (r + 2.0) ** 3) * c["F"] * 4
+        if l > 0 and acc + b > 32 * 2**20:
+            lo.append(l)
+            acc = 0.0
+        acc += b
+    return lo + [c["L"]]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed", range(8))
+def test_random_level_groups(seed):
+    """The level-major schedule on tables of 2^19 and 2^20 entries, whose levels fall into
+    several groups of different sizes: indices, forward, fp32 and fp16 gradients against
+    the oracle."""
+    import multiresolution_hash_grid_b200 as hg
+    c = level_config(seed)
+    L, F, log2T, n = c["L"], c["F"], c["log2T"], c["n"]
+    f16 = c["dtype"] == "f16"
+    grid = hg.HashGrid(L, F, log2T, c["N_min"], c["N_max"], hg.HASHGRID_F16 if f16 else hg.HASHGRID_F32,
+                       forward_gather=GATHER[c["gather"]], backward_mode=BACKWARD[c["backward"]],
+                       schedule=SCHEDULE["level"])
+    og = oracle.Grid(L, F, log2T, c["N_min"], c["N_max"], oracle.F16 if f16 else oracle.F32)
+    rng = np.random.default_rng(8000 + seed)
+    table = workloads.table_values(rng, L, 2**log2T, F, c["dtype"])
+    x = rng.random((n, 3), dtype=np.float32)
+    k = min(n, 8)
+    x[:k] = EDGE[rng.integers(0, len(EDGE), size=(k, 3))]
+    g = workloads.upstream_grads(rng, n, L * F)
+    x_d, t_d, g_d = dev(x), dev(table), dev(g)
+    np.testing.assert_array_equal(grid.indices(x_d).cpu().numpy().view(np.uint32), og.indices(x), err_msg=str(c))
+    out = grid.forward(x_d, t_d).cpu().numpy().astype(np.float64)
+    ref = og.forward(x, table, nthreads=THREADS)
+    bound = og.forward(x, np.abs(table), nthreads=THREADS)
+    assert np.all(np.abs(out - ref) <= FWD_RTOL[c["dtype"]] * bound + 1e-30), c
+    got = grid.backward(x_d, g_d).cpu().numpy()
+    check_gradient(got, og.backward(x, g, nthreads=THREADS))
+    dh = torch.zeros((L, 2**log2T, F), dtype=torch.float16, device="cuda")
+    hg.hashgrid_backward_half(grid.handle, x_d, g_d, n, dh)
+    torch.cuda.synchronize()
+    check_half_gradient(og, x, g, dh.cpu().numpy())
+
+
+def test_level_group_configurations_have_several_groups():
+    """Host check: every level-major seed splits its levels into at least two groups, and
+    the seeds include groups of more than one level."""
+    gs = [level_groups(level_config(s)) for s in range(8)]
+    assert all(len(g) >= 3 for g in gs), gs
+    assert any(max(b - a for a, b in zip(g, g[1:])) > 1 for g in gs), gs
